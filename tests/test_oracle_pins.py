@@ -1,0 +1,308 @@
+"""Pins of the fp64 CPU oracle to facts outside itself (CPU only).
+
+Each check targets a part of the oracle with a value fixed by the mathematics or the pages, so that a
+plausible slip (a dropped scale, a wrong sign, a transposed operand, an off-by-one causal mask, a
+wrong LSE base, a bad group merge) fails at least one of them:
+
+  * hand-derived worked examples (tests/golden/hand_examples.json);
+  * Q = 0 closed form: O is the mean of the visible V rows, LSE = ln(#visible keys);
+  * causal row 0: O_0 = V_0, LSE_0 = scale * q_0 . k_0;
+  * a library softmax / logsumexp (scipy) applied to the same scores;
+  * key-shift invariance: K + 1 c^T leaves O unchanged and shifts LSE by scale * q . c;
+  * joint permutation of K and V rows leaves non-causal results unchanged (position independence
+    of exact attention, "Was FlashAttention bei Transformer-Inference verändert");
+  * linearity in V;
+  * scalar brute force (math.fsum) on tiny inputs, all mask kinds;
+  * the tiled online-softmax loop and the 3-group merge of "轻松读懂FlashAttention 上" against the
+    materialised definition;
+  * padded + 2-D key mask against packed varlen (to rounding, on valid rows);
+  * split-KV partials + combine against the materialised single-query result;
+  * safe softmax: huge scores stay finite ("小知识" note under "内存卡点").
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+import seeded_inputs as si
+
+RTOL = 1e-12
+
+
+def rnd(shape, seed, dtype="bf16"):
+    bits = si.normal_bits([99, seed], int(np.prod(shape)), dtype)
+    return si.bits_to_float(bits, dtype).reshape(shape)
+
+
+# ---------------------------------------------------------------------------------------------
+# hand-derived golden cases
+
+
+def _f(x):
+    return -math.inf if x == "-inf" else float(x)
+
+
+def _golden_cases(golden_dir):
+    with open(os.path.join(golden_dir, "hand_examples.json")) as fh:
+        return json.load(fh)["cases"]
+
+
+def test_hand_examples_materialised(golden_dir):
+    for c in _golden_cases(golden_dir):
+        o, lse = oracle.attention_head(np.array(c["q"]), np.array(c["k"]), np.array(c["v"]),
+                                       c["scale"], c["causal"])
+        np.testing.assert_allclose(o, np.array(c["o"]), rtol=0, atol=1e-13, err_msg=c["name"])
+        exp_lse = np.array([_f(x) for x in c["lse"]])
+        assert np.array_equal(np.isinf(lse), np.isinf(exp_lse)), c["name"]
+        fin = np.isfinite(exp_lse)
+        np.testing.assert_allclose(lse[fin], exp_lse[fin], rtol=0, atol=1e-13, err_msg=c["name"])
+
+
+def test_hand_examples_brute_and_tiled(golden_dir):
+    for c in _golden_cases(golden_dir):
+        exp_o = np.array(c["o"])
+        exp_lse = np.array([_f(x) for x in c["lse"]])
+        bo, bl = oracle.brute_attention_head(c["q"], c["k"], c["v"], c["scale"], c["causal"])
+        to, tl = oracle.tiled_online_attention(np.array(c["q"]), np.array(c["k"]), np.array(c["v"]),
+                                               c["scale"], c["causal"], block_q=2, block_k=2)
+        for o, lse in ((np.array(bo), np.array(bl)), (to, tl)):
+            np.testing.assert_allclose(o, exp_o, rtol=0, atol=1e-13, err_msg=c["name"])
+            fin = np.isfinite(exp_lse)
+            assert np.array_equal(np.isfinite(lse), fin), c["name"]
+            np.testing.assert_allclose(lse[fin], exp_lse[fin], rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# closed forms
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_closed_form(causal):
+    n, d = 37, 8
+    q = np.zeros((n, d))
+    k = rnd((n, d), 1)
+    v = rnd((n, d), 2)
+    o, lse = oracle.attention_head(q, k, v, scale=0.3, causal=causal)
+    for i in range(n):
+        vis = i + 1 if causal else n
+        np.testing.assert_allclose(o[i], v[:vis].mean(axis=0), rtol=RTOL, atol=1e-14)
+        assert abs(lse[i] - math.log(vis)) < 1e-13
+
+
+def test_causal_row_zero_closed_form():
+    n, d = 20, 16
+    q, k, v = rnd((n, d), 3), rnd((n, d), 4), rnd((n, d), 5)
+    scale = 0.125
+    o, lse = oracle.attention_head(q, k, v, scale, causal=True)
+    np.testing.assert_array_equal(o[0], v[0])
+    assert abs(lse[0] - scale * float(np.dot(q[0], k[0]))) < 1e-13
+
+
+def test_single_key_returns_value_row():
+    q, k, v = rnd((5, 4), 6), rnd((1, 4), 7), rnd((1, 3), 8)
+    o, lse = oracle.attention_head(q, k, v, 0.7)
+    np.testing.assert_array_equal(o, np.repeat(v, 5, axis=0))
+    np.testing.assert_allclose(lse, 0.7 * (q @ k[0]), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------------------------
+# library routines
+
+
+@pytest.mark.parametrize("scale", [0.125, 1.0 / math.sqrt(128), 0.1])
+def test_matches_scipy_softmax_noncausal(scale):
+    nq, nk, d, dv = 19, 23, 16, 12
+    q, k, v = rnd((nq, d), 9), rnd((nk, d), 10), rnd((nk, dv), 11)
+    o, lse = oracle.attention_head(q, k, v, scale)
+    scores = scale * np.einsum("id,jd->ij", q, k)
+    np.testing.assert_allclose(o, scipy.special.softmax(scores, axis=1) @ v, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, scipy.special.logsumexp(scores, axis=1), rtol=1e-13)
+
+
+def test_matches_scipy_softmax_causal_rectangular():
+    nq, nk, d = 7, 12, 8
+    q, k, v = rnd((nq, d), 12), rnd((nk, d), 13), rnd((nk, d), 14)
+    o, lse = oracle.attention_head(q, k, v, 0.4, causal=True)
+    for i in range(nq):
+        last = i + (nk - nq) + 1
+        sc = 0.4 * np.array([np.dot(q[i], k[j]) for j in range(last)])
+        np.testing.assert_allclose(o[i], scipy.special.softmax(sc) @ v[:last], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse[i], scipy.special.logsumexp(sc), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# invariants
+
+
+def test_key_shift_invariance():
+    nq, nk, d = 9, 15, 8
+    q, k, v = rnd((nq, d), 15), rnd((nk, d), 16), rnd((nk, d), 17)
+    c = rnd((d,), 18)
+    scale = 0.37
+    o1, l1 = oracle.attention_head(q, k, v, scale)
+    o2, l2 = oracle.attention_head(q, k + c[None, :], v, scale)
+    np.testing.assert_allclose(o2, o1, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(l2, l1 + scale * (q @ c), rtol=1e-12, atol=1e-12)
+
+
+def test_joint_key_value_permutation_invariance():
+    nq, nk, d = 11, 29, 8
+    q, k, v = rnd((nq, d), 19), rnd((nk, d), 20), rnd((nk, d), 21)
+    perm = np.random.default_rng(0).permutation(nk)
+    o1, l1 = oracle.attention_head(q, k, v, 0.2)
+    o2, l2 = oracle.attention_head(q, k[perm], v[perm], 0.2)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l2, l1, rtol=1e-13)
+
+
+def test_linear_in_values():
+    nq, nk, d = 6, 10, 4
+    q, k = rnd((nq, d), 22), rnd((nk, d), 23)
+    v1, v2 = rnd((nk, 5), 24), rnd((nk, 5), 25)
+    a = rnd((5, 3), 26)
+    o1, _ = oracle.attention_head(q, k, v1, 0.5, causal=True)
+    o2, _ = oracle.attention_head(q, k, v2, 0.5, causal=True)
+    o12, _ = oracle.attention_head(q, k, v1 + v2, 0.5, causal=True)
+    oa, _ = oracle.attention_head(q, k, v1 @ a, 0.5, causal=True)
+    np.testing.assert_allclose(o12, o1 + o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(oa, o1 @ a, rtol=1e-12, atol=1e-13)
+
+
+def test_safe_softmax_stays_finite():
+    q = np.array([[1.0, 0.0], [0.0, 1.0]])
+    k = np.array([[3000.0, 0.0], [2990.0, 1.0], [0.0, 5000.0]])
+    v = np.array([[1.0], [2.0], [3.0]])
+    o, lse = oracle.attention_head(q, k, v, 1.0)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    # row 0: scores 3000, 2990, 0 -> weights ~ (1, e^-10, 0)
+    w = np.array([1.0, math.exp(-10.0)])
+    np.testing.assert_allclose(o[0, 0], (w @ [1.0, 2.0]) / w.sum(), rtol=1e-14)
+    np.testing.assert_allclose(lse[0], 3000.0 + math.log(w.sum()), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------------------------
+# brute force on tiny inputs
+
+
+@pytest.mark.parametrize("nq,nk,causal,k_valid", [
+    (1, 1, False, None), (4, 4, True, None), (5, 9, True, None), (9, 5, True, None),
+    (16, 16, False, 11), (7, 13, False, None), (16, 16, True, None), (3, 16, False, 1),
+])
+def test_matches_brute_force(nq, nk, causal, k_valid):
+    d, dv = 6, 5
+    q, k, v = rnd((nq, d), 30 + nq), rnd((nk, d), 40 + nk), rnd((nk, dv), 50 + nk)
+    o, lse = oracle.attention_head(q, k, v, 0.3, causal, k_valid)
+    bo, bl = oracle.brute_attention_head(q.tolist(), k.tolist(), v.tolist(), 0.3, causal, k_valid)
+    bo, bl = np.array(bo), np.array(bl)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-14)
+    assert np.array_equal(np.isfinite(lse), np.isfinite(bl))
+    fin = np.isfinite(bl)
+    np.testing.assert_allclose(lse[fin], bl[fin], rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# the tiled algorithm and the group merge against the definition
+
+
+@pytest.mark.parametrize("nq,nk,causal,bq,bk,k_valid", [
+    (300, 300, True, 128, 128, None), (300, 300, False, 128, 128, None),
+    (257, 513, True, 64, 128, None), (129, 77, True, 32, 16, None),
+    (200, 200, False, 128, 128, 133), (64, 64, True, 64, 64, None),
+])
+def test_tiled_online_matches_materialised(nq, nk, causal, bq, bk, k_valid):
+    d = 16
+    q, k, v = rnd((nq, d), 60), rnd((nk, d), 61), rnd((nk, d), 62)
+    o, lse = oracle.attention_head(q, k, v, 0.25, causal, k_valid)
+    to, tl = oracle.tiled_online_attention(q, k, v, 0.25, causal, bq, bk, k_valid)
+    np.testing.assert_allclose(to, o, rtol=1e-12, atol=1e-13)
+    fin = np.isfinite(lse)
+    assert np.array_equal(np.isfinite(tl), fin)
+    np.testing.assert_allclose(tl[fin], lse[fin], rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("n,groups", [(3, 3), (10, 3), (100, 3), (1000, 7), (5, 5)])
+def test_group_merge_equals_full_softmax(n, groups):
+    x = 3.0 * rnd((n,), 70 + n)
+    p, m, l = oracle.softmax_by_groups(x, groups)
+    np.testing.assert_allclose(p, scipy.special.softmax(x), rtol=1e-12, atol=1e-300)
+    assert m == x.max()
+    np.testing.assert_allclose(m + math.log(l), scipy.special.logsumexp(x), rtol=1e-14)
+
+
+def test_group_merge_order_independent_of_max_position():
+    x = np.array([0.0, 1.0, 50.0, -3.0, 2.0, 49.5])
+    p_a, _, _ = oracle.softmax_by_groups(x, 3)
+    p_b, _, _ = oracle.softmax_by_groups(x, 2)
+    p_c, _, _ = oracle.softmax_by_groups(x, 6)
+    np.testing.assert_allclose(p_a, p_b, rtol=1e-14)
+    np.testing.assert_allclose(p_a, p_c, rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# varlen / key padding
+
+
+def test_padded_key_mask_equals_packed_varlen():
+    lengths = [5, 17, 1, 12]
+    H, D = 2, 8
+    q, k, v, cu = si.varlen_qkv(7, lengths, H, D, "fp16")
+    qf, kf, vf = (si.bits_to_float(t, "fp16") for t in (q, k, v))
+    o_p, l_p = oracle.attention_varlen(qf, kf, vf, cu, 0.1)
+    nmax = max(lengths)
+    B = len(lengths)
+    pad = lambda t: np.stack([np.pad(t[cu[b]:cu[b + 1]], ((0, nmax - lengths[b]), (0, 0), (0, 0)),
+                                     constant_values=7.0) for b in range(B)])
+    mask = np.array([[j < lengths[b] for j in range(nmax)] for b in range(B)])
+    o_d, l_d = oracle.padded_key_mask_attention(pad(qf), pad(kf), pad(vf), mask, 0.1)
+    for b in range(B):
+        L = lengths[b]
+        # equal up to the summation order of the BLAS products (padded rows change the blocking)
+        np.testing.assert_allclose(o_d[b, :L], o_p[cu[b]:cu[b + 1]], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(l_d[b, :, :L], l_p[:, cu[b]:cu[b + 1]], rtol=1e-14, atol=1e-14)
+
+
+def test_varlen_key_valid_equals_truncation():
+    n, d = 40, 8
+    q, k, v = rnd((n, d), 80), rnd((n, d), 81), rnd((n, d), 82)
+    o1, l1 = oracle.attention_head(q, k, v, 0.3, k_valid=23)
+    o2, l2 = oracle.attention_head(q, k[:23], v[:23], 0.3)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# decode: split-KV partials + combine
+
+
+@pytest.mark.parametrize("nk,splits", [(64, 1), (64, 16), (100, 16), (37, 3), (5, 16), (8192, 16)])
+def test_split_kv_combine_equals_full(nk, splits):
+    d = 32
+    q, k, v = rnd((d,), 90), rnd((nk, d), 91), rnd((nk, d), 92)
+    scale = 1.0 / math.sqrt(d)
+    o_ref, l_ref = oracle.attention_head(q[None, :], k, v, scale)
+    parts_o, parts_l = oracle.split_kv_partials(q, k, v, scale, splits)
+    o, lse = oracle.combine_partials(parts_o, parts_l)
+    np.testing.assert_allclose(o, o_ref[0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, l_ref[0], rtol=1e-13)
+    # each partial is itself the attention over its own key range
+    for s, (lo, hi) in enumerate(oracle.online.split_bounds(nk, splits)):
+        if hi > lo:
+            po, pl = oracle.attention_head(q[None, :], k[lo:hi], v[lo:hi], scale)
+            np.testing.assert_allclose(parts_o[s], po[0], rtol=1e-12, atol=1e-14)
+        else:
+            assert parts_l[s] == -np.inf
+
+
+def test_row_sampler_matches_full_head():
+    nq, nk, d = 70, 70, 8
+    q, k, v = rnd((nq, d), 93), rnd((nk, d), 94), rnd((nk, d), 95)
+    rows = [0, 1, 33, 69]
+    for causal in (False, True):
+        o, lse = oracle.attention_head(q, k, v, 0.5, causal)
+        ro, rl = oracle.attention_rows(q, k, v, rows, 0.5, causal)
+        np.testing.assert_allclose(ro, o[rows], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(rl, lse[rows], rtol=1e-13)
