@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the exact tiled attention forward pass on B200; prints ONE JSON line (rank 0).
+
+Headline: attention forward TFLOPS on the prefill workload B=4, H=16, N=8192, D=64, causal, bf16
+(4*B*H*N^2*D FLOPs, halved for causal), inputs resident in HBM.  One step = one fa_fwd call over the
+whole batch.  The same line carries
+  * roofline  -- the prefill kernel's achieved TFLOP/s against the measured dense bf16 peak;
+  * decode    -- split-KV decode (B=64, H=32, D=128, Nk=8192, 16 splits) in HBM GB/s of K+V+Q+O
+                 bytes, with its own roofline against the measured HBM copy bandwidth;
+  * e2e       -- the same headline metric through the C ABI with host buffers: every step copies
+                 Q, K, V from pinned host memory and O, LSE back;
+  * cpu_baseline -- the fp64 CPU oracle on a bounded sample of the workload (rank 0, N=1 only);
+  * clocks    -- SM clocks and throttle reasons sampled (NVML) during the timed region.
+
+--impl reference times the CPU oracle itself as the reference arm (rank 0 only).
+Multi-GPU (--gpus N under torchrun): one process per GPU, each rank runs its own batch of the same
+workload (independent problems, no data-path collective); value = all ranks' FLOPs / max-over-ranks
+time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import seeded_inputs as si  # noqa: E402
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE = "prefill_d64"
+METRIC = "attention fwd TFLOPS (and % of B200 dense bf16 peak); decode HBM GB/s"
+
+
+def peaks():
+    try:
+        with open(MEASURED_PEAKS) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def prefill_flops(B, H, Nq, Nk, D, causal):
+    f = 4.0 * B * H * Nq * Nk * D
+    return f / 2 if causal else f
+
+
+def causal_rows_flops(rows_lo, rows_hi, N, D):
+    """Algorithmic FLOPs of query rows [lo, hi) of one causal head with Nq = Nk = N."""
+    # row i sees i+1 keys: 4 * (i+1) * D
+    n = rows_hi - rows_lo
+    s = (rows_lo + 1 + rows_hi) * n / 2.0
+    return 4.0 * D * s
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU with NVML every ~20 ms (read-only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# device helpers
+
+
+def to_dev(bits, dtype, device):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device)
+    return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+
+
+def timed(fn, steps, stream, dist=None):
+    """Time `steps` calls of fn on `stream` with CUDA events; returns (ms total, max over ranks)."""
+    import torch
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle legs
+
+
+def oracle_prefill_sample(cfg, budget_s, head_iter=None):
+    """Run the fp64 oracle on the last rows of heads of the prefill workload for ~budget_s seconds.
+
+    The last r query rows of a causal head with all N keys are exactly those rows of the full
+    problem (bottom-right alignment).  Returns (flops, seconds, description).
+    """
+    import oracle
+    B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
+    causal = cfg.get("causal", False)
+    # one batch item's tensors on the host (regenerated from the seed, as on the GPU side)
+    b = 0
+    qb = si.batch_item(cfg["seed"], si.Q_ID, b, (N, H, D), dt)
+    kb = si.batch_item(cfg["seed"], si.K_ID, b, (N, H, D), dt)
+    vb = si.batch_item(cfg["seed"], si.V_ID, b, (N, H, D), dt)
+    rows = 256
+    flops = 0.0
+    t0 = time.perf_counter()
+    heads = 0
+    while True:
+        h = heads % H
+        qf = si.bits_to_float(qb[N - rows:, h], dt)
+        kf = si.bits_to_float(kb[:, h], dt)
+        vf = si.bits_to_float(vb[:, h], dt)
+        oracle.attention_head(qf, kf, vf, cfg["scale"], causal)
+        flops += causal_rows_flops(N - rows, N, N, D) if causal else 4.0 * rows * N * D
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return flops, el, f"fp64 oracle on the last {rows} query rows of {heads} head(s) of batch item 0"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the oracle as the program being compared against
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = si.CONFIGS[HEADLINE]
+    total_budget = 90.0
+    per_step = max(0.05, total_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_prefill_sample(cfg, per_step)
+    flops = secs = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        f, s, desc = oracle_prefill_sample(cfg, per_step)
+        flops += f
+        secs += s
+    tflops = flops / secs / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": HEADLINE, "B": cfg["B"], "H": cfg["H"], "N": cfg["Nq"], "D": cfg["D"],
+                   "causal": True, "input_dtype": cfg["dtype"]},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import exact_tiled_attention_47_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist = tdist
+    fa._lib.load()
+    pk, pk_kind = peaks()
+
+    # ---------------- prefill headline ----------------
+    cfg = si.CONFIGS[HEADLINE]
+    B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
+    seed = cfg["seed"] + 1000 * rank  # each rank: its own batch of the same workload
+    q, k, v = si.dense_qkv(seed, B, N, N, H, D, dt)
+    qd, kd, vd = (to_dev(t, dt, dev) for t in (q, k, v))
+    od = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = cfg["scale"]
+
+    def step():
+        st = fa.fa_fwd(qd, kd, vd, od, lse, B, H, N, N, D, scale, True, None, stream)
+        if st:
+            raise fa.FAError(st, "fa_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed(step, args.steps, stream, dist)
+    if fa.fa_device_status(clear=True) != 0:
+        raise RuntimeError("device status set during the timed prefill run")
+    flops_step = prefill_flops(B, H, N, N, D, True)
+    ms_step = ms / args.steps
+    tflops_rank = flops_step / (ms_step * 1e-3) / 1e12
+    value = tflops_rank * world
+    peak_b, peak_s = pk["bf16_tflops"], pk["bf16_tflops_sustained"]
+    roof = {"bound": "tensor", "achieved": tflops_rank, "peak": peak_b, "unit": "TFLOP/s",
+            "frac": tflops_rank / peak_b, "traffic": None,
+            "kernel": "fa_fwd_kernel<64,bf16,out bf16>",
+            "peak_kind": f"{pk_kind} bf16 burst", "frac_of_sustained": tflops_rank / peak_s,
+            "algorithmic_flops_per_launch": flops_step}
+
+    # ---------------- e2e through the C ABI with host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (torch.from_numpy(np.ascontiguousarray(t).view(np.int16)).view(torch.bfloat16).pin_memory()
+                      for t in (q, k, v))
+        oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+        lh = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 30))
+        for _ in range(2):
+            e2e_step()
+        ms_e2e = timed(e2e_step, e2e_steps, stream, dist)
+        h2d = 3 * qh.numel() * 2
+        d2h = oh.numel() * 2 + lh.numel() * 4
+        e2e = {"value": flops_step * world / (ms_e2e / e2e_steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": ms_e2e / e2e_steps}
+        del qh, kh, vh, oh, lh
+    del qd, kd, vd, od, lse
+    torch.cuda.empty_cache()
+
+    # ---------------- decode (secondary metric) ----------------
+    dec = None
+    if not args.no_decode:
+        c = si.CONFIGS["decode"]
+        Bd, Hd, Nk, Dd, S = c["B"], c["H"], c["Nk"], c["D"], c["num_splits"]
+        dseed = c["seed"] + 1000 * rank
+        qd_ = to_dev(si.batched(dseed, si.Q_ID, Bd, (1, Hd, Dd), "bf16"), "bf16", dev)
+        kc = torch.empty((Bd, Nk, Hd, Dd), dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        for b in range(Bd):  # chunked upload keeps host memory bounded
+            kc[b].copy_(to_dev(si.batch_item(dseed, si.K_ID, b, (Nk, Hd, Dd), "bf16"), "bf16", dev))
+            vc[b].copy_(to_dev(si.batch_item(dseed, si.V_ID, b, (Nk, Hd, Dd), "bf16"), "bf16", dev))
+        o_ = torch.empty_like(qd_)
+        l_ = torch.empty((Bd, Hd), dtype=torch.float32, device=dev)
+        wsb = fa.fa_decode_workspace_bytes(Bd, Hd, Dd, S)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        dscale = c["scale"]
+
+        def dstep():
+            st = fa.fa_decode_splitkv(qd_, kc, vc, o_, l_, Bd, Hd, Nk, Dd, dscale, S, ws, wsb, stream)
+            if st:
+                raise fa.FAError(st, "fa_decode_splitkv")
+
+        for _ in range(args.warmup):
+            dstep()
+        dsteps = max(10, args.steps // 2)
+        ms_d = timed(dstep, dsteps, stream, dist)
+        if fa.fa_device_status(clear=True) != 0:
+            raise RuntimeError("device status set during the timed decode run")
+        kv_bytes = 2 * Bd * Nk * Hd * Dd * 2
+        alg_bytes = kv_bytes + 2 * Bd * Hd * Dd * 2 + Bd * Hd * 4
+        gbs = alg_bytes / (ms_d / dsteps * 1e-3) / 1e9
+        dec = {"metric": "decode HBM GB/s", "value": gbs * world, "unit": "GB/s",
+               "ms_per_step": ms_d / dsteps, "steps": dsteps,
+               "config": {"workload": "decode", "B": Bd, "H": Hd, "Nk": Nk, "D": Dd, "num_splits": S,
+                          "dtype": "bf16", "l2": "K/V cache 8.6 GB > L2"},
+               "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                            "peak_kind": f"{pk_kind} copy", "algorithmic_bytes_per_step": alg_bytes},
+               "gpu_launches": 2 * dsteps}
+        del qd_, kc, vc, o_, l_, ws
+        torch.cuda.empty_cache()
+
+    # ---------------- CPU baseline (oracle) ----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        f, s, desc = oracle_prefill_sample(cfg, args.cpu_budget)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "seconds": s}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": HEADLINE, "B": B, "H": H, "N": N, "D": D, "causal": True,
+                   "input_dtype": dt, "output_dtype": "bf16", "scale": scale,
+                   "l2": "inputs 192 MiB > 126 MB L2 (no flush needed)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": args.steps,
+        "decode": dec, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+"""Exact tiled attention for NVIDIA B200 (sm_100a): Python binding of libfa_sm100.so.
+
+The functions named like the C entry points (``fa_fwd``, ``fa_decode_splitkv``, ...) only marshal
+arguments -- tensors become device pointers, torch streams become ``cudaStream_t`` -- and return the
+C status code.  ``attention`` and ``decode`` additionally allocate the outputs with torch and raise
+``FAError`` on a non-zero status.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU path.  PyTorch supplies device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+from ._lib import LIB_PATH, LibraryMissing, SIGNATURES, load
+
+FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
+(FA_OK, FA_ERR_NULL, FA_ERR_DTYPE, FA_ERR_HEADDIM, FA_ERR_SHAPE, FA_ERR_ALIGN, FA_ERR_CU_SEQLENS,
+ FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT) = range(11)
+
+__all__ = [
+    "fa_fwd", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_status_string",
+    "fa_device_status", "fa_abi_version", "attention", "decode", "FAError", "LibraryMissing",
+    "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
+]
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({fa_status_string(status)})")
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.bfloat16: FA_BF16, torch.float16: FA_FP16, torch.float32: FA_FP32}.get(t.dtype, -1)
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu_seqlens=None, stream=None,
+           in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_fwd``; returns its status.  Dtypes default to those of q and o."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    return lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(H), int(Nq), int(Nk),
+                      int(D), float(scale), int(bool(causal)), _ptr(cu_seqlens), _stream(stream),
+                      int(in_dtype), int(o_dtype))
+
+
+def fa_decode_workspace_bytes(B, H, D, num_splits) -> int:
+    return int(load().fa_decode_workspace_bytes(int(B), int(H), int(D), int(num_splits)))
+
+
+def fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace,
+                      workspace_bytes=None, stream=None, in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_splitkv``; returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), int(B),
+                                 int(H), int(Nk), int(D), float(scale), int(num_splits),
+                                 _ptr(workspace), int(workspace_bytes), _stream(stream),
+                                 int(in_dtype), int(o_dtype))
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def fa_device_status(clear: bool = True) -> int:
+    """Device status word of the current device (synchronises); resets it when ``clear``."""
+    out = ctypes.c_int(-1)
+    st = load().fa_device_status(ctypes.byref(out), int(bool(clear)))
+    if st != FA_OK:
+        raise FAError(st, "fa_device_status")
+    return out.value
+
+
+def fa_abi_version() -> int:
+    return int(load().fa_abi_version())
+
+
+# ------------------------------------------------------------------------------------------------
+# allocating helpers (torch allocates; the library computes)
+
+
+def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None, stream=None):
+    """O, LSE for q [B,Nq,H,D], k/v [B,Nk,H,D] (dense) or packed [total,H,D] with cu_seqlens."""
+    import torch
+    D = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if cu_seqlens is None:
+        B, Nq, H, _ = q.shape
+        Nk = k.shape[1]
+        lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
+    else:
+        Nq, H, _ = q.shape
+        Nk = k.shape[0]
+        B = cu_seqlens.numel() - 1
+        lse = torch.empty((H, Nq), device=q.device, dtype=torch.float32)
+    o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
+    st = fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu_seqlens, stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, workspace=None,
+           stream=None):
+    """O [B,1,H,D], LSE [B,H] for one query per (batch, head) over the cache [B,Nk,H,D]."""
+    import torch
+    B, _, H, D = q.shape
+    Nk = k_cache.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    nbytes = fa_decode_workspace_bytes(B, H, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
+    lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    st = fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace,
+                           workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_decode_splitkv")
+    return o, lse

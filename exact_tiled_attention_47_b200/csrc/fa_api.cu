@@ -1,0 +1,210 @@
+// fa_api.cu -- the extern "C" boundary of libfa_sm100.so (declared in include/fa.h).
+//
+// Argument checks run on the host before anything is enqueued, in a fixed order: null pointers,
+// element types, head dimension, shapes and scale, alignment, workspace, then the device.  Kernels
+// report failures they detect (a bounded wait that ran out, an inconsistent cu_seqlens) through a
+// per-device status word read by fa_device_status().
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+__device__ int g_status_word = 0;
+
+constexpr int kMaxDevices = 64;
+int g_device_ok[kMaxDevices];      // 0 unknown, 1 sm_100, -1 other
+int* g_status_ptr[kMaxDevices];
+std::mutex g_mu;
+
+}  // namespace
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// FA_OK if the current device is an sm_100 part, else FA_ERR_DEVICE.
+int check_device(int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_device_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_DEVICE;
+    }
+    g_device_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_device_ok[dev] == 1 ? FA_OK : FA_ERR_DEVICE;
+}
+
+int* device_status_ptr() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace fa
+
+extern "C" {
+
+int fa_abi_version(void) { return 1; }
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "a required pointer is NULL";
+    case FA_ERR_DTYPE: return "unsupported element type (inputs must be bf16 or fp16; output the input type or fp32)";
+    case FA_ERR_HEADDIM: return "unsupported head dimension (must be 64 or 128)";
+    case FA_ERR_SHAPE: return "invalid shape, split count or scale";
+    case FA_ERR_ALIGN: return "a tensor pointer is misaligned (16 bytes; lse 4 bytes)";
+    case FA_ERR_CU_SEQLENS: return "cu_seqlens is not non-decreasing within the packed extent";
+    case FA_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case FA_ERR_DEVICE: return "no usable sm_100 (B200) CUDA device";
+    case FA_ERR_LAUNCH: return "CUDA launch or driver call failed";
+    case FA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    default: return "unknown status";
+  }
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+           int D, float scale, int causal, const int* cu_seqlens, fa_stream_t stream, int in_dtype,
+           int o_dtype) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
+  if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
+  if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || H > 65535) return FA_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (cu_seqlens) {
+    if (Nq != Nk) return FA_ERR_SHAPE;  // self-attention: one packed extent for Q and K/V
+    if (static_cast<int64_t>(Nq) / 128 + B > INT32_MAX) return FA_ERR_SHAPE;
+  } else {
+    if (B > 65535 || Nq > (1 << 24) || Nk > (1 << 24)) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(B) * Nq >= INT32_MAX || static_cast<int64_t>(B) * Nk >= INT32_MAX)
+      return FA_ERR_SHAPE;
+  }
+  if (!fa::aligned(q, 16) || !fa::aligned(k, 16) || !fa::aligned(v, 16) || !fa::aligned(o, 16) || !fa::aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if (cu_seqlens && !fa::aligned(cu_seqlens, 4)) return FA_ERR_ALIGN;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  int* status = fa::device_status_ptr();
+  if (!status) return FA_ERR_LAUNCH;
+  fa::PrefillArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.cu_seqlens = cu_seqlens;
+  a.status = status;
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.D = D;
+  a.scale = scale;
+  a.causal = causal != 0;
+  a.fp16 = in_dtype == FA_FP16;
+  a.o_fp32 = o_dtype == FA_FP32;
+  const int e = fa::launch_prefill(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != 0) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
+size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits) {
+  if (B < 1 || H < 1 || num_splits < 1 || (D != 64 && D != 128)) return 0;
+  const size_t n = static_cast<size_t>(num_splits) * B * H;
+  const size_t bytes = n * D * sizeof(float) + n * sizeof(float);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
+                      int H, int Nk, int D, float scale, int num_splits, void* workspace,
+                      size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype) {
+  if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_NULL;
+  if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
+  if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
+  if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || Nk < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
+  if (num_splits < 1 || num_splits > 128) return FA_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * H > (static_cast<int64_t>(1) << 28)) return FA_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (!fa::aligned(q, 16) || !fa::aligned(k_cache, 16) || !fa::aligned(v_cache, 16) || !fa::aligned(o, 16) || !fa::aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < fa_decode_workspace_bytes(B, H, D, num_splits)) return FA_ERR_WORKSPACE;
+  if (!fa::aligned(workspace, 16)) return FA_ERR_ALIGN;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  int* status = fa::device_status_ptr();
+  if (!status) return FA_ERR_LAUNCH;
+  fa::DecodeArgs a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.lse = lse;
+  const size_t n = static_cast<size_t>(num_splits) * B * H;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_lse = static_cast<float*>(workspace) + n * D;
+  a.status = status;
+  a.B = B;
+  a.H = H;
+  a.Nk = Nk;
+  a.D = D;
+  a.S = num_splits;
+  a.scale = scale;
+  a.fp16 = in_dtype == FA_FP16;
+  a.o_fp32 = o_dtype == FA_FP32;
+  const int e = fa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != 0) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
+int fa_device_status(int* status_out, int clear) {
+  if (!status_out) return FA_ERR_NULL;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  int* p = fa::device_status_ptr();
+  if (!p) return FA_ERR_LAUNCH;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  *status_out = v;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// fa_internal.h -- launchers shared between the C-ABI layer (fa_api.cu) and the kernel files.
+// Arguments reaching these functions have already been validated.
+#pragma once
+#include <cstddef>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int* cu_seqlens;  // nullptr = dense mode
+  int* status;            // device status word
+  int B, H, Nq, Nk, D;
+  float scale;
+  int causal;
+  int fp16;    // input type: 1 = fp16, 0 = bf16
+  int o_fp32;  // output type: 1 = fp32, 0 = input type
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  float* ws_o;    // [B, H, S, D]
+  float* ws_lse;  // [B, H, S]
+  int* status;
+  int B, H, Nk, D, S;
+  float scale;
+  int fp16;
+  int o_fp32;
+};
+
+// Return a cudaError_t-compatible code (0 = success).
+int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+int* device_status_ptr();  // address of this device's status word (nullptr on failure)
+
+}  // namespace fa

@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact tiled attention library (libfa_sm100.so).
+ *
+ * What it computes.  O = softmax(scale * Q K^T + mask) V for every (batch, head), together with the
+ * per-row natural log-sum-exp LSE_i = ln sum_j exp(scale * q_i . k_j) over the visible keys j.  The
+ * three steps of standard attention (scores, row softmax, product with V) are those of the Ascend
+ * CANN ops-transformer FlashAttention article (zskr.cn), section "背景"; the tiled evaluation with a
+ * running row max m and running row sum l is its section "原理" (steps 1-4).  The result is exact
+ * attention, not an approximation ("Was FlashAttention bei Transformer-Inference verändert"): the
+ * N x N matrices S and P never leave the chip and are never returned (output_attentions has no
+ * counterpart, as in the parameter table of "如何为 Hugging Face Transformers 更多架构添加 Flash
+ * Attention 2 支持？").
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named q, k, v, o, k_cache, v_cache, lse, cu_seqlens and workspace are DEVICE
+ *     pointers of the current CUDA device.  The caller owns every buffer; the library never
+ *     allocates, frees or synchronises.  All work is enqueued on `stream` (0 = legacy default
+ *     stream) and runs asynchronously.
+ *   - Q/K/V/O layout is [B, N, H, D], row-major and contiguous (the layout of the tiling sketch in
+ *     the Ascend article, section "代码讲解").  Element types: FA_BF16 or FA_FP16 inputs; the
+ *     output O is either the input type or FA_FP32.  LSE is always fp32.
+ *   - Head dimension D must be 64 or 128 (the Hugging Face page asks for a head_dim of at least 64
+ *     that is a multiple of 64 / a power of two; these are the two sizes the kernels implement).
+ *   - fp32/fp64 inputs are rejected with FA_ERR_DTYPE (Hugging Face page, "常见错误排查", error 1).
+ *   - Only sm_100 devices (B200) are accepted; anything else returns FA_ERR_DEVICE (same page,
+ *     error 3, states the GPU-generation gate).
+ *   - Every argument is validated before anything is launched; on error nothing is enqueued and the
+ *     status code is returned.  No entry point aborts, throws or prints.
+ *   - Device-side failures (a bounded wait inside a kernel that ran out) are recorded in a device
+ *     status word that fa_device_status() reads.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                     /* the same type as cudaStream_t */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1, FA_FP32 = 2 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = 1,        /* a required pointer is NULL                                      */
+  FA_ERR_DTYPE = 2,       /* input not bf16/fp16, or output type not (input type | fp32)      */
+  FA_ERR_HEADDIM = 3,     /* D not in {64, 128}                                               */
+  FA_ERR_SHAPE = 4,       /* B, H, Nq, Nk, num_splits out of range, or scale not finite > 0   */
+  FA_ERR_ALIGN = 5,       /* a tensor pointer is not 16-byte aligned (lse: 4-byte)            */
+  FA_ERR_CU_SEQLENS = 6,  /* cu_seqlens inconsistent with the packed extent (device-detected) */
+  FA_ERR_WORKSPACE = 7,   /* decode workspace missing or smaller than required                */
+  FA_ERR_DEVICE = 8,      /* no CUDA device, or the current device is not sm_100             */
+  FA_ERR_LAUNCH = 9,      /* a CUDA launch or driver call failed                              */
+  FA_ERR_TIMEOUT = 10     /* a bounded wait inside a kernel ran out (device-detected)         */
+} fa_status;
+
+/*
+ * fa_fwd -- attention forward pass over many queries (prefill / encoder).
+ *
+ * Passage: Ascend article sections "原理" (tiling, online softmax with m and l) and "代码讲解"
+ * (outer loop over query blocks, inner loop over key/value blocks); the mask kinds of the Hugging
+ * Face page ("原因分析" item 1: causal and bidirectional; "常见错误排查" error 4: the 2-D key
+ * padding mask) and its varlen variant (FAQ 4, flash_attn_varlen).
+ *
+ * Dense mode (cu_seqlens == NULL):
+ *   q [B, Nq, H, D], k and v [B, Nk, H, D], o [B, Nq, H, D] of type o_dtype, lse [B, H, Nq].
+ * Varlen mode (cu_seqlens != NULL): B sequences packed back to back,
+ *   q, k, v, o [total, H, D] with total = Nq = Nk (the packed row extent of the buffers);
+ *   cu_seqlens: device int32[B + 1], cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = total;
+ *   sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 and its queries see exactly its own
+ *   keys (self-attention: one cu_seqlens for Q and K); lse [H, total].  The kernels never touch a
+ *   row outside [0, total).  A cu_seqlens that is not non-decreasing or ends above total is
+ *   detected on the device: its tiles are skipped and the device status becomes FA_ERR_CU_SEQLENS.
+ * causal != 0: query i (0-based within its sequence) sees key j iff j <= i + (Nk_b - Nq_b),
+ *   i.e. the lower triangle aligned at the bottom-right corner; with Nq_b = Nk_b this is j <= i.
+ *   A query that sees no key gets O = 0 and LSE = -inf.
+ * scale: the softmax scale, finite and > 0 (callers wanting the default pass 1/sqrt(D)).
+ * in_dtype: FA_BF16 or FA_FP16; o_dtype: in_dtype or FA_FP32.
+ * Limits: 1 <= B, 1 <= H, 1 <= Nq, Nk <= 2^24 rows per batch item (dense) or packed (varlen);
+ *   B * Nq and B * Nk below 2^31.
+ * Returns FA_OK or an fa_status error code; see the conventions above.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int Nq, int Nk, int D, float scale, int causal,
+           const int* cu_seqlens, fa_stream_t stream, int in_dtype, int o_dtype);
+
+/*
+ * fa_decode_workspace_bytes -- size of the scratch buffer fa_decode_splitkv needs:
+ * num_splits * B * H * (D + 1) * 4 bytes (one fp32 partial output row and one fp32 partial LSE per
+ * split), rounded up to 256 bytes.  Returns 0 for invalid arguments.
+ */
+size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits);
+
+/*
+ * fa_decode_splitkv -- single-token decode over a KV cache with split-KV and an LSE combine.
+ *
+ * Passage: "Was FlashAttention bei Transformer-Inference verändert" (prefill versus decode of a
+ * single token differ in the parallel work available; the cache layout question), and the merge of
+ * per-group softmax statistics of "轻松读懂FlashAttention 上", section "Softmax求解重构", which is
+ * exactly how the per-split partial results are combined.
+ *
+ * q [B, 1, H, D]; k_cache, v_cache [B, Nk, H, D]; o [B, 1, H, D] of type o_dtype; lse [B, H].
+ * The query attends to all Nk cached keys (no mask).  The keys are cut into num_splits ranges of
+ * ceil(Nk / num_splits) keys; a first kernel writes each range's normalised partial output and
+ * partial LSE to `workspace`, a second kernel merges them.  1 <= num_splits <= 128.
+ * workspace: device buffer of at least fa_decode_workspace_bytes(B, H, D, num_splits) bytes, owned
+ * by the caller, 16-byte aligned; its contents on entry are irrelevant.
+ * Returns FA_OK or an fa_status error code.
+ */
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                      int B, int H, int Nk, int D, float scale, int num_splits,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream,
+                      int in_dtype, int o_dtype);
+
+/* fa_status_string -- static English text for a status code (never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * fa_device_status -- read the device status word of the current device into *status_out
+ * (FA_OK if no kernel recorded a failure) and, if clear != 0, reset it to FA_OK.  This call
+ * synchronises with the device (it copies one int).  Returns FA_OK, FA_ERR_NULL, FA_ERR_DEVICE or
+ * FA_ERR_LAUNCH.
+ */
+int fa_device_status(int* status_out, int clear);
+
+/* fa_abi_version -- version of this interface (incremented on any signature change). */
+int fa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

@@ -1,0 +1,143 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every symbol declared in
+include/*.h, and rejects bad arguments with the documented status codes before touching a device.
+
+Fake pointers are used only in cases that fail validation before the device check, so no test here
+can ever reach a kernel launch, with or without a GPU.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import exact_tiled_attention_47_b200 as fa
+from exact_tiled_attention_47_b200 import build as fabuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fabuild.build()
+    return fa._lib.load()
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(fa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("fa_fwd", "fa_decode_splitkv", "fa_decode_workspace_bytes", "fa_status_string",
+              "fa_device_status", "fa_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+        assert n in fa._lib.SIGNATURES, f"binding has no signature for {n}"
+
+
+def test_binding_names_match_c_names():
+    for n in _declared_functions():
+        assert callable(getattr(fa, n)), n
+
+
+def test_abi_version_and_status_strings(lib):
+    assert fa.fa_abi_version() == 1
+    seen = set()
+    for code in range(11):
+        s = fa.fa_status_string(code)
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 11
+    assert fa.fa_status_string(999) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    B, H, D, S = 64, 32, 128, 16
+    exp = S * B * H * (D + 1) * 4
+    got = fa.fa_decode_workspace_bytes(B, H, D, S)
+    assert got >= exp and got % 256 == 0 and got - exp < 256
+    assert fa.fa_decode_workspace_bytes(0, H, D, S) == 0
+    assert fa.fa_decode_workspace_bytes(B, H, 96, S) == 0
+    assert fa.fa_decode_workspace_bytes(B, H, D, 0) == 0
+
+
+A = 0x100000  # a 16-byte aligned fake address (never dereferenced: every case fails validation)
+
+
+def _fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, Nq=128, Nk=128, D=64, scale=0.125, causal=0,
+         cu=None, in_dtype=0, o_dtype=0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu, None, in_dtype, o_dtype)
+
+
+def test_fwd_validation_codes(lib):
+    assert _fwd(lib, q=None) == fa.FA_ERR_NULL
+    assert _fwd(lib, lse=None) == fa.FA_ERR_NULL
+    assert _fwd(lib, in_dtype=2) == fa.FA_ERR_DTYPE          # fp32 inputs rejected
+    assert _fwd(lib, in_dtype=5) == fa.FA_ERR_DTYPE
+    assert _fwd(lib, in_dtype=0, o_dtype=1) == fa.FA_ERR_DTYPE  # bf16 in, fp16 out
+    assert _fwd(lib, D=32) == fa.FA_ERR_HEADDIM
+    assert _fwd(lib, D=96) == fa.FA_ERR_HEADDIM
+    assert _fwd(lib, D=256) == fa.FA_ERR_HEADDIM
+    assert _fwd(lib, B=0) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, Nk=0) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, Nq=0) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, scale=0.0) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, scale=-1.0) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, scale=float("nan")) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, scale=float("inf")) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, B=70000) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, B=200, Nq=1 << 24) == fa.FA_ERR_SHAPE
+    assert _fwd(lib, cu=A, Nq=100, Nk=200) == fa.FA_ERR_SHAPE  # varlen needs one packed extent
+    assert _fwd(lib, q=A + 8) == fa.FA_ERR_ALIGN
+    assert _fwd(lib, o=A + 2) == fa.FA_ERR_ALIGN
+    assert _fwd(lib, lse=A + 2) == fa.FA_ERR_ALIGN
+    assert _fwd(lib, cu=A + 2) == fa.FA_ERR_ALIGN
+
+
+def _dec(lib, q=A, k=A, v=A, o=A, lse=A, B=2, H=2, Nk=64, D=128, scale=0.1, S=4, ws=A,
+         wsb=1 << 20, in_dtype=0, o_dtype=0):
+    return lib.fa_decode_splitkv(q, k, v, o, lse, B, H, Nk, D, scale, S, ws, wsb, None, in_dtype, o_dtype)
+
+
+def test_decode_validation_codes(lib):
+    assert _dec(lib, k=None) == fa.FA_ERR_NULL
+    assert _dec(lib, in_dtype=2) == fa.FA_ERR_DTYPE
+    assert _dec(lib, o_dtype=1) == fa.FA_ERR_DTYPE
+    assert _dec(lib, D=80) == fa.FA_ERR_HEADDIM
+    assert _dec(lib, Nk=0) == fa.FA_ERR_SHAPE
+    assert _dec(lib, S=0) == fa.FA_ERR_SHAPE
+    assert _dec(lib, S=129) == fa.FA_ERR_SHAPE
+    assert _dec(lib, scale=0.0) == fa.FA_ERR_SHAPE
+    assert _dec(lib, v=A + 4) == fa.FA_ERR_ALIGN
+    assert _dec(lib, ws=None) == fa.FA_ERR_WORKSPACE
+    need = fa.fa_decode_workspace_bytes(2, 2, 128, 4)
+    assert _dec(lib, wsb=need - 1) == fa.FA_ERR_WORKSPACE
+    assert _dec(lib, ws=A + 8, wsb=need) == fa.FA_ERR_ALIGN
+
+
+def test_device_status_null(lib):
+    assert lib.fa_device_status(None, 0) == fa.FA_ERR_NULL
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU answer")
+def test_no_device_is_reported(lib):
+    # All arguments valid: the only failing check is the device one, and nothing is launched.
+    assert _fwd(lib) == fa.FA_ERR_DEVICE
+    assert _dec(lib) == fa.FA_ERR_DEVICE
+    out = ctypes.c_int(0)
+    assert lib.fa_device_status(ctypes.byref(out), 0) == fa.FA_ERR_DEVICE
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(fa.LibraryMissing):
+        fa._lib.load(str(tmp_path / "nope.so"))
