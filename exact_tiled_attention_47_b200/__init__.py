@@ -19,7 +19,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 
 __all__ = [
     "fa_fwd", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_status_string",
-    "fa_device_status", "fa_abi_version", "attention", "decode", "FAError", "LibraryMissing",
+    "fa_device_status", "fa_abi_version", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
 
@@ -83,6 +83,29 @@ def fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_split
                                  int(H), int(Nk), int(D), float(scale), int(num_splits),
                                  _ptr(workspace), int(workspace_bytes), _stream(stream),
                                  int(in_dtype), int(o_dtype))
+
+
+# Size of the library's fixed decode scratch array (FA_NOALLOC_SCRATCH_BYTES in include/fa.h).
+FA_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def fa_decode_splitkv_noalloc(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits,
+                              stream=None, in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_splitkv_noalloc``: decode for callers that cannot allocate.
+
+    Same results as ``fa_decode_splitkv``; the split partials live in the library's fixed
+    per-GPU scratch array instead of a caller workspace, so nothing is allocated per call.
+    Calls on one device share that array: do not let two of them overlap on the GPU.
+    """
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    return lib.fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                         int(B), int(H), int(Nk), int(D), float(scale),
+                                         int(num_splits), _stream(stream), int(in_dtype),
+                                         int(o_dtype))
 
 
 def fa_status_string(status: int) -> str:

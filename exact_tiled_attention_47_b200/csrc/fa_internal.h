@@ -2,6 +2,7 @@
 // Arguments reaching these functions have already been validated.
 #pragma once
 #include <cstddef>
+#include <cstdint>
 #include <cuda_runtime.h>
 
 namespace fa {
@@ -41,5 +42,7 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 int* device_status_ptr();  // address of this device's status word (nullptr on failure)
+int check_device(int* dev_out);  // FA_OK if the current device is sm_100, else FA_ERR_DEVICE
+bool aligned(const void* p, uintptr_t a);
 
 }  // namespace fa

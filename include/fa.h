@@ -115,6 +115,29 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, v
                       void* workspace, size_t workspace_bytes, fa_stream_t stream,
                       int in_dtype, int o_dtype);
 
+/*
+ * fa_decode_splitkv_noalloc -- fa_decode_splitkv without a caller-provided workspace.
+ *
+ * The pages describe nothing like this; it exists for callers that cannot allocate device memory
+ * when they call: an engine that reserves all of its memory at start-up and forbids allocation
+ * afterwards, a plugin whose host framework owns the allocator, or latency-critical code that must
+ * not pay for cudaMalloc (which can synchronise the device).  Arguments, layouts and results are
+ * those of fa_decode_splitkv minus workspace/workspace_bytes.  The per-split partials go to a fixed
+ * array of FA_NOALLOC_SCRATCH_BYTES inside the library, reserved on each GPU where the library's
+ * code is first used and kept until the process exits.
+ *   - Returns FA_ERR_WORKSPACE, without launching, when fa_decode_workspace_bytes(B, H, D,
+ *     num_splits) exceeds FA_NOALLOC_SCRATCH_BYTES.
+ *   - The first call on a device looks up the array's device address (with that device current)
+ *     and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Nothing in it needs clearing between calls, but
+ *     calls whose kernels may overlap on the GPU (unordered streams) race on it: order them.
+ *   - Calls no allocating routine (no cudaMalloc / cudaFree).
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                              int B, int H, int Nk, int D, float scale, int num_splits,
+                              fa_stream_t stream, int in_dtype, int o_dtype);
+
 /* fa_status_string -- static English text for a status code (never NULL). */
 const char* fa_status_string(int status);
 
