@@ -243,49 +243,16 @@ def run_reference(args):
 # our arm
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
-    if args.impl == "reference":
-        return run_reference(args)
-
-    import torch
-    import exact_tiled_attention_47_b200 as fa
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as tdist
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        dist = tdist
-    fa._lib.load()
-    pk, pk_kind = peaks()
-
-    # ---------------- prefill headline ----------------
-    cfg = si.CONFIGS[HEADLINE]
+def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
+    """Time the headline prefill workload; returns (value, ms_step, roofline, e2e, clocks)."""
     B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
+    scale = cfg["scale"]
+    stream = torch.cuda.current_stream(dev)
     seed = cfg["seed"] + 1000 * rank  # each rank: its own batch of the same workload
     q, k, v = si.dense_qkv(seed, B, N, N, H, D, dt)
     qd, kd, vd = (to_dev(t, dt, dev) for t in (q, k, v))
     od = torch.empty_like(qd)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    scale = cfg["scale"]
 
     def step():
         st = fa.fa_fwd(qd, kd, vd, od, lse, B, H, N, N, D, scale, True, None, stream)
@@ -295,7 +262,7 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         ms = timed(step, args.steps, stream, dist)
     if fa.fa_device_status(clear=True) != 0:
         raise RuntimeError("device status set during the timed prefill run")
@@ -339,11 +306,66 @@ def main():
     del qd, kd, vd, od, lse
     torch.cuda.empty_cache()
 
+    return value, ms_step, roof, e2e, clk
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="profiling runs: time only one of the two paths")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="profiling runs: smaller decode batch than the workload's B=64")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import exact_tiled_attention_47_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist = tdist
+    fa._lib.load()
+    pk, pk_kind = peaks()
+
+    # ---------------- prefill headline ----------------
+    cfg = si.CONFIGS[HEADLINE]
+    run_prefill = args.only in ("all", "prefill")
+    run_decode = args.only in ("all", "decode") and not args.no_decode
+    B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
+    scale = cfg["scale"]
+    stream = torch.cuda.current_stream(dev)
+    value = ms_step = None
+    roof = e2e = None
+    clk = ClockSampler(local)
+    if run_prefill:
+        value, ms_step, roof, e2e, clk = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch)
+
     # ---------------- decode (secondary metric) ----------------
     dec = None
-    if not args.no_decode:
+    if run_decode:
         c = si.CONFIGS["decode"]
         Bd, Hd, Nk, Dd, S = c["B"], c["H"], c["Nk"], c["D"], c["num_splits"]
+        if args.decode_batch:
+            Bd = args.decode_batch
         dseed = c["seed"] + 1000 * rank
         qd_ = to_dev(si.batched(dseed, si.Q_ID, Bd, (1, Hd, Dd), "bf16"), "bf16", dev)
         kc = torch.empty((Bd, Nk, Hd, Dd), dtype=torch.bfloat16, device=dev)
@@ -374,7 +396,7 @@ def main():
         dec = {"metric": "decode HBM GB/s", "value": gbs * world, "unit": "GB/s",
                "ms_per_step": ms_d / dsteps, "steps": dsteps,
                "config": {"workload": "decode", "B": Bd, "H": Hd, "Nk": Nk, "D": Dd, "num_splits": S,
-                          "dtype": "bf16", "l2": "K/V cache 8.6 GB > L2"},
+                          "dtype": "bf16", "l2": f"K/V cache {kv_bytes / 1e9:.2f} GB vs 126 MB L2"},
                "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                             "frac": gbs / pk["hbm_gbs"], "traffic": None,
                             "peak_kind": f"{pk_kind} copy", "algorithmic_bytes_per_step": alg_bytes},
@@ -384,7 +406,7 @@ def main():
 
     # ---------------- CPU baseline (oracle) ----------------
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and run_prefill:
         f, s, desc = oracle_prefill_sample(cfg, args.cpu_budget)
         cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": desc, "seconds": s}
@@ -402,7 +424,8 @@ def main():
                    "input_dtype": dt, "output_dtype": "bf16", "scale": scale,
                    "l2": "inputs 192 MiB > 126 MB L2 (no flush needed)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": args.steps,
+        "roofline": roof, "clocks": clk.summary(), "e2e": e2e,
+        "gpu_launches": args.steps if run_prefill else 0,
         "decode": dec, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
