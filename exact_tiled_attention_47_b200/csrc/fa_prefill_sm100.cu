@@ -5,20 +5,29 @@
 // block scores, keep a running row max m and row sum l, rescale the output accumulator when m grows,
 // add P_j V_j, and divide by l at the end.  S and P never leave the chip.
 //
-// Mapping to sm_100a (one CTA per 128-row Q tile of one (batch, head)):
-//   warp 0      TMA producer: the Q tile once, then K_j and V_j through a kStages-deep ring of
-//               128-byte-swizzled shared-memory tiles tracked by mbarriers.
-//   warp 1      owns the tensor memory and issues the tensor-core work from one thread:
-//               S_j = Q K_j^T  (tcgen05.mma, both operands in shared memory, fp32 into TMEM), and
-//               O  += P_j V_j  (tcgen05.mma, P read from TMEM, V from shared memory).
-//               S is double-buffered in TMEM so S_{j+1} runs while the softmax works on S_j.
-//   warps 2..5  softmax: thread r owns query row r (TMEM lane r).  It reads its 128 scores with
-//               tcgen05.ld, applies the causal / key-length mask, updates m and l, computes
-//               P = 2^(S*scale*log2(e) - m) with the MUFU ex2, rescales its O row in TMEM when m
-//               grew, writes P (bf16/fp16) back to TMEM, and finally writes O / l and the LSE.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P [384,448) (P packs two 16-bit values per
-// 32-bit column).  Causal runs stop at the last key block that the tile's last row can see, so
-// fully masked blocks are never loaded or multiplied.
+// Mapping to sm_100a.  One CTA owns two 128-row Q tiles (256 rows) of one (batch, head), so every
+// K/V tile brought into shared memory feeds both, and the tensor core alternates between the tiles
+// while the other tile's softmax runs ("ping-pong"):
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r of a warpgroup owns query
+//               row r (TMEM lane r).  Per key block it reads its 128 scores with tcgen05.ld, masks
+//               them (causal diagonal / key-length tail only), updates the running max m and sum l,
+//               computes P = 2^(S*scale*log2(e) - m) -- part of the exponentials on the MUFU unit,
+//               part with a polynomial on the FMA pipe -- writes P (bf16/fp16) to TMEM, and at the end
+//               writes O / l and the LSE.  O is rescaled only when m grew by more than 2^8 since the
+//               last rescale; until then P and l use the stale max, which is exact because O and l
+//               share it.
+//   warp 8      TMA producer: Q tiles once, then K_j and V_j through rings of 128-byte-swizzled
+//               shared-memory stages tracked by mbarriers.
+//   warp 9      owns the tensor memory and issues every tcgen05.mma from one thread, in the order
+//               S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...  The commit that signals S_t(j+1)
+//               covers all earlier MMAs, so it also tells softmax t that PV_t(j) is done (its P
+//               buffer is free and O_t is stable).
+//   warps 10-11 idle.
+// TMEM (512 columns): S0 [0,128) S1 [128,256); D=64: O0 [256,320) O1 [320,384) P0 [384,448)
+// P1 [448,512); D=128: O0 [256,384) O1 [384,512) and P_t in the upper half of S_t (P is written
+// only after the whole S row was read; the next S_t is issued after the PV_t that reads P_t).
+// Causal runs stop at the last key block the tile's last row can see; fully masked blocks are never
+// loaded or multiplied.  Work units are issued longest first.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -30,35 +39,57 @@ namespace fa {
 namespace {
 
 constexpr int kBM = 128;  // query rows per tile
-constexpr int kBN = 128;  // keys per tile
-constexpr int kThreads = 192;
+constexpr int kBN = 128;  // keys per block
+constexpr int kTiles = 2;
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
 constexpr int kPanelBytes = kBM * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P and O may grow by up to 2^8
 constexpr uint64_t kDrainLimitNs = 200000000ull;
+// Registers: launched with kLaunchRegs per thread; the two softmax warpgroups then take
+// kSoftmaxRegs and the producer/MMA warpgroup gives back down to kControlRegs.  The split must not
+// exceed the launch allocation (256 * 216 + 128 * 72 = 384 * 168), else setmaxnreg.inc would wait
+// forever; the host refuses to launch if the compiled register count differs from kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
+constexpr int kEmuEvery = 8;  // of every kEmuEvery column pairs ...
+#ifndef FA_EMU_PAIRS
+#define FA_EMU_PAIRS 3
+#endif
+constexpr int kEmuPairs = FA_EMU_PAIRS;  // ... this many take the polynomial exp2
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kTileBytes = kBM * D * 2;
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kKStages = (D == 64) ? 4 : 2;
+  static constexpr int kVStages = (D == 64) ? 4 : 2;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kKOff = kQOff + kTiles * kTileBytes;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
+  __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
+  __device__ static constexpr uint32_t col_o(int t) { return t ? ((D == 64) ? 320u : 384u) : 256u; }
+  __device__ static constexpr uint32_t col_p(int t) {
+    return t ? ((D == 64) ? 448u : 192u) : ((D == 64) ? 384u : 64u);
+  }
 };
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, o_done, drain;
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  int tile_b, tile_m;
+  int tile_b, tile_pair;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
 
@@ -68,6 +99,7 @@ struct FwdParams {
   const int* cu;
   int* status;
   int B, H, Nq, Nk;
+  int num_pairs;  // dense: ceil(Nq / 256)
   float scale_log2;
   int causal;
 };
@@ -88,9 +120,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-// Varlen: map a linear tile slot to (sequence, row block) by a warp-wide scan of the tile counts.
-__device__ void find_varlen_tile(const FwdParams& p, int lane, int& out_b, int& out_m) {
-  const int tile = blockIdx.x;
+// Varlen: map a linear slot to (sequence, 256-row pair) by a warp-wide scan of per-sequence counts.
+__device__ void find_varlen_pair(const FwdParams& p, int slot, int lane, int& out_b, int& out_pair) {
   const int total = p.Nq;
   int base = 0, fb = -1, fm = -1;
   bool bad = false;
@@ -102,7 +133,7 @@ __device__ void find_varlen_tile(const FwdParams& p, int lane, int& out_b, int& 
       if (lo < 0 || hi < lo || hi > total) bad = true;
       else len = hi - lo;
     }
-    const int nt = (len + kBM - 1) / kBM;
+    const int nt = (len + kTiles * kBM - 1) / (kTiles * kBM);
     int incl = nt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -110,19 +141,64 @@ __device__ void find_varlen_tile(const FwdParams& p, int lane, int& out_b, int& 
       if (lane >= o) incl += t;
     }
     const int excl = incl - nt;
-    const bool mine = nt > 0 && tile >= base + excl && tile < base + incl;
+    const bool mine = nt > 0 && slot >= base + excl && slot < base + incl;
     const unsigned bal = __ballot_sync(0xffffffffu, mine);
     if (bal != 0u) {
       const int src = __ffs(bal) - 1;
       fb = c + src;
-      fm = tile - base - __shfl_sync(0xffffffffu, excl, src);
+      fm = slot - base - __shfl_sync(0xffffffffu, excl, src);
       break;
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(p.status, kStatusCuSeqlens);
   out_b = fb;
-  out_m = fm;
+  out_pair = fm;
+}
+
+// O and LSE of rows that see no key at all.
+template <int D, bool kOutF32>
+__device__ void write_empty_row(const FwdParams& p, int b, int h, int q_row0, int qi) {
+  const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
+  if constexpr (kOutF32) {
+    float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow);
+    for (int d = 0; d < D / 4; ++d) out[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow);
+    for (int d = 0; d < D / 8; ++d) out[d] = make_uint4(0, 0, 0, 0);
+  }
+  const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
+                                      : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
+  p.lse[li] = -INFINITY;
+}
+
+// P for 32 score columns (chunk ch of the row): x = s * scale * log2(e) - m, p = 2^x (on the MUFU
+// unit, or -- for kEmuPairs of every kEmuEvery column pairs when kMixed -- by the FMA-pipe
+// polynomial), row-sum accumulation in two packed fp32 chains, conversion to the input type and a
+// 16-column TMEM store (two 16-bit values per column).
+template <bool kMixed, bool kFp16>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[128], int ch, uint64_t sl2x2, uint64_t negm,
+                                          uint64_t& acc0, uint64_t& acc1, uint32_t p_addr) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = ch * 32 + 2 * i;
+    const uint64_t x = f2_fma(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
+    uint64_t pe;
+    if (kMixed && (i % kEmuEvery) < kEmuPairs) {
+      pe = exp2_poly_pair(x);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      pe = f2(ex2(x0), ex2(x1));
+    }
+    if (i & 1) acc1 = f2_add(acc1, pe);
+    else acc0 = f2_add(acc0, pe);
+    float p0, p1;
+    f2_split(pe, p0, p1);
+    pk[i] = pack2<kFp16>(p0, p1);
+  }
+  tmem_st16(p_addr + ch * 16, pk);
 }
 
 template <int D, bool kFp16, bool kOutF32>
@@ -136,25 +212,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
 
-  // ---- tile geometry --------------------------------------------------------------------------
-  int b, m_block;
+  // ---- work unit: (b, h, pair of Q tiles) -----------------------------------------------------
+  int b, h, pair;
   if (p.cu == nullptr) {
-    b = blockIdx.z;
-    m_block = blockIdx.x;
+    const int bh_count = p.B * p.H;
+    const int bh = blockIdx.x % bh_count;
+    pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x / bh_count);  // longest (causal) first
+    b = bh / p.H;
+    h = bh % p.H;
   } else {
+    h = blockIdx.x % p.H;
+    const int slot = blockIdx.x / p.H;
     if (warp == 0) {
       int fb, fm;
-      find_varlen_tile(p, lane, fb, fm);
+      find_varlen_pair(p, slot, lane, fb, fm);
       if (lane == 0) {
         bars->tile_b = fb;
-        bars->tile_m = fm;
+        bars->tile_pair = fm;
       }
     }
     __syncthreads();
     b = bars->tile_b;
-    m_block = bars->tile_m;
+    pair = bars->tile_pair;
     if (b < 0) return;  // spare slot (uniform across the CTA)
   }
   int q_row0, k_row0, Lq, Lk;
@@ -167,52 +247,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     q_row0 = k_row0 = p.cu[b];
     Lq = Lk = p.cu[b + 1] - p.cu[b];
   }
-  const int m0 = m_block * kBM;
-  int kv_end = Lk;
-  if (p.causal) kv_end = min(Lk, m0 + kBM + (Lk - Lq));
-  const int n_kv = kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
-
-  if (n_kv == 0) {  // no row of this tile sees any key: O = 0, LSE = -inf
-    if (warp >= 2) {
-      const int r = (warp & 3) * 32 + lane;
-      const int qi = m0 + r;
-      if (qi < Lq) {
-        const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
-        if constexpr (kOutF32) {
-          float* out = static_cast<float*>(p.o) + orow;
-          for (int d = 0; d < D; d += 4) *reinterpret_cast<float4*>(out + d) = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          uint16_t* out = static_cast<uint16_t*>(p.o) + orow;
-          for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4*>(out + d) = make_uint4(0, 0, 0, 0);
-        }
-        const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
-                                            : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
-        p.lse[li] = -INFINITY;
-      }
-    }
-    return;
+  const int m0 = pair * (kTiles * kBM);
+  const int diag = Lk - Lq;  // bottom-right causal alignment
+  int n_kv[kTiles];
+#pragma unroll
+  for (int t = 0; t < kTiles; ++t) {
+    const int first = m0 + t * kBM;
+    int kv_end = Lk;
+    if (p.causal) kv_end = min(Lk, first + kBM + diag);
+    n_kv[t] = (first < Lq && kv_end > 0) ? (kv_end + kBN - 1) / kBN : 0;
   }
+  const int n_max = max(n_kv[0], n_kv[1]);
+
+  // softmax warps of tiles without any visible key write O = 0, LSE = -inf directly
+  if (warp < 8) {
+    const int t = warp >> 2;
+    if (n_kv[t] == 0) {
+      const int qi = m0 + t * kBM + (warp & 3) * 32 + lane;
+      if (qi < Lq) write_empty_row<D, kOutF32>(p, b, h, q_row0, qi);
+    }
+  }
+  if (n_max == 0) return;  // uniform
 
   // ---- setup ----------------------------------------------------------------------------------
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 4);
+      mbar_init(&bars->o_done[t], 1);
+    }
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 4);
-    }
-    mbar_init(&bars->p_full, 4);
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -222,216 +299,246 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
 
-  uint8_t* sQ = smem + C::kQOff;
+  auto sQ = [&](int t) { return smem + C::kQOff + t * C::kTileBytes; };
   auto sK = [&](int st) { return smem + C::kKOff + st * C::kTileBytes; };
   auto sV = [&](int st) { return smem + C::kVOff + st * C::kTileBytes; };
 
-  if (warp == 0) {
+  if (warp >= 8) {
+    regs_decrease<kControlRegs>();
+  if (warp == kProducerWarp) {
     // ================================ TMA producer ===============================================
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
       const uint64_t keep = l2_policy_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
+      for (int t = 0; t < kTiles; ++t) {
+        if (n_kv[t] == 0) continue;
+        mbar_arrive_expect_tx(&bars->q_full[t], C::kTileBytes);
 #pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_3d(&tmap_q, &bars->q_full, sQ + pn * kPanelBytes, pn * 64, h, q_row0 + m0);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(&tmap_q, &bars->q_full[t], sQ(t) + pn * kPanelBytes, pn * 64, h, q_row0 + m0 + t * kBM);
+      }
       int last_k[4] = {-1, -1, -1, -1}, last_v[4] = {-1, -1, -1, -1};
       bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!(ok = mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag, p.status))) break;
-        mbar_arrive_expect_tx(&bars->k_full[st], C::kTileBytes);
+      for (int j = 0; j < n_max; ++j) {
+        const int ks = j % C::kKStages, vs = j % C::kVStages;
+        if (!(ok = mbar_wait(&bars->k_empty[ks], ((j / C::kKStages) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&bars->k_full[ks], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d_hint(&tmap_k, &bars->k_full[st], sK(st) + pn * kPanelBytes, pn * 64, h,
-                           k_row0 + j * kBN, keep);
-        last_k[st] = j;
-        if (!(ok = mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag, p.status))) break;
-        mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes);
+          tma_load_3d_hint(&tmap_k, &bars->k_full[ks], sK(ks) + pn * kPanelBytes, pn * 64, h, k_row0 + j * kBN, keep);
+        last_k[ks] = j;
+        if (!(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVStages) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d_hint(&tmap_v, &bars->v_full[st], sV(st) + pn * kPanelBytes, pn * 64, h,
-                           k_row0 + j * kBN, keep);
-        last_v[st] = j;
+          tma_load_3d_hint(&tmap_v, &bars->v_full[vs], sV(vs) + pn * kPanelBytes, pn * 64, h, k_row0 + j * kBN, keep);
+        last_v[vs] = j;
       }
       if (!ok) {  // let every copy this thread started land before the CTA exits
-        drain_wait(&bars->q_full, 0);
-        for (int st = 0; st < C::kStages; ++st) {
-          if (last_k[st] >= 0) drain_wait(&bars->k_full[st], (last_k[st] / C::kStages) & 1);
-          if (last_v[st] >= 0) drain_wait(&bars->v_full[st], (last_v[st] / C::kStages) & 1);
-        }
+        for (int t = 0; t < kTiles; ++t)
+          if (n_kv[t] > 0) drain_wait(&bars->q_full[t], 0);
+        for (int st = 0; st < C::kKStages; ++st)
+          if (last_k[st] >= 0) drain_wait(&bars->k_full[st], (last_k[st] / C::kKStages) & 1);
+        for (int st = 0; st < C::kVStages; ++st)
+          if (last_v[st] >= 0) drain_wait(&bars->v_full[st], (last_v[st] / C::kVStages) & 1);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ================================ MMA issuer =================================================
     if (lane == 0) {
       constexpr int fmt = kFp16 ? 0 : 1;
       constexpr uint32_t idesc_qk = instr_desc_f16(kBM, kBN, fmt, 0);
       constexpr uint32_t idesc_pv = instr_desc_f16(kBM, D, fmt, 1);
-      const uint32_t sQa = smem_addr(sQ);
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!mbar_wait(&bars->k_full[st], ph, abort_flag, p.status)) return false;
-        if (j >= 2 && !mbar_wait(&bars->s_free[j & 1], ((j >> 1) - 1) & 1, abort_flag, p.status))
-          return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tbase + ((j & 1) ? kColS1 : kColS0);
-        const uint32_t sKa = smem_addr(sK(st));
+      bool ok = true;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t sQa = smem_addr(sQ(t));
+        const uint32_t sKa = smem_addr(sK(j % C::kKStages));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row;
           // every 4 steps move to the next 64-column panel.  SBO = 8 rows * 128 B.
           const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(sQa + off, 16, 1024), smem_desc_sw128(sKa + off, 16, 1024),
+          mma_ss(tbase + C::col_s(t), smem_desc_sw128(sQa + off, 16, 1024), smem_desc_sw128(sKa + off, 16, 1024),
                  idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->s_full[j & 1]);
-        mma_commit(&bars->k_empty[st]);
-        return true;
+        mma_commit(&bars->s_full[t]);
       };
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i % C::kStages;
-        const uint32_t ph = (i / C::kStages) & 1;
-        if (!mbar_wait(&bars->v_full[st], ph, abort_flag, p.status)) return false;
-        if (!mbar_wait(&bars->p_full, i & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t sVa = smem_addr(sV(st));
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t sVa = smem_addr(sV(j % C::kVStages));
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // V is N-major (head dim contiguous): 16 keys = two 8-row swizzle atoms = 2048 bytes;
           // LBO = distance between the 64-column panels, SBO = 8 rows * 128 B.
-          mma_ts(tbase + kColO, tbase + kColP + kk * 8, smem_desc_sw128(sVa + kk * 2048, kPanelBytes, 1024),
-                 idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tbase + C::col_o(t), tbase + C::col_p(t) + kk * 8,
+                 smem_desc_sw128(sVa + kk * 2048, kPanelBytes, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bars->o_done);
-        mma_commit(&bars->v_empty[st]);
-        return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 1; ok && j <= n_kv; ++j) {
-        if (j < n_kv) ok = issue_s(j);
-        if (ok) ok = issue_pv(j - 1);
+      // prologue: S_t(0) for both tiles
+      for (int t = 0; t < kTiles && ok; ++t)
+        if (n_kv[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, p.status);
+      if (ok) ok = mbar_wait(&bars->k_full[0], 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < kTiles; ++t)
+          if (n_kv[t] > 0) issue_s(t, 0);
+        mma_commit(&bars->k_empty[0]);
+      }
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int vs = j % C::kVStages;
+        if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
+        const bool next = j + 1 < n_max;
+        bool k_next_ready = false;
+        for (int t = 0; t < kTiles; ++t) {
+          if (j >= n_kv[t]) continue;
+          if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          if (j + 1 < n_kv[t]) {
+            if (!k_next_ready) {
+              const int ks = (j + 1) % C::kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(t, j + 1);
+          } else {
+            mma_commit(&bars->o_done[t]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->v_empty[vs]);
+        if (next) {
+          if (!k_next_ready) {  // no tile needed K(j+1): still hand the stage back in order
+            const int ks = (j + 1) % C::kKStages;
+            if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
+          }
+          mma_commit(&bars->k_empty[(j + 1) % C::kKStages]);
+        }
       }
       // no tensor-core work may still be in flight when TMEM and shared memory are released
       mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
     }
+  }
   } else {
-    // ================================ softmax / correction / epilogue ============================
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int qi = m0 + r;
-    const int diag = Lk - Lq;  // bottom-right causal alignment
-    const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;      // keys [0,row_lim) visible
-    const int tile_lim = p.causal ? min(Lk, m0 + 1 + diag) : Lk;     // smallest row_lim of the tile
-    const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!(ok = warp_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, p.status))) break;
-      tc_fence_after();
-      const uint32_t s_addr = lane_base + ((j & 1) ? kColS1 : kColS0);
-      uint32_t sr[128];
-      tmem_ld128_sync(s_addr, sr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[j & 1]);
-
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      if ((j + 1) * kBN > tile_lim) {
-        const int lim = row_lim - j * kBN;
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m_run - m_use);
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(s[c], sl2, -m_use));
-        const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c >> 1] = pack2<kFp16>(p0, p1);
-      }
-      l_run = l_run * alpha + (rs0 + rs1);
-      if (j > 0) {
-        // PV of the previous block must be done: it reads the P buffer and accumulates into O.
-        if (!(ok = warp_wait(&bars->o_done, (j - 1) & 1, abort_flag, p.status))) break;
+    regs_increase<kSoftmaxRegs>();
+    // ================================ softmax / epilogue =========================================
+    const int t = warp >> 2;
+    const int n = n_kv[t];
+    if (n > 0) {
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;
+      const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int tile_m0 = m0 + t * kBM;
+      const int qi = tile_m0 + r;
+      const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;         // keys [0,row_lim) visible
+      const int tile_lim = p.causal ? min(Lk, tile_m0 + 1 + diag) : Lk;   // smallest row_lim of the tile
+      const float sl2 = p.scale_log2;
+      const uint64_t sl2x2 = f2(sl2, sl2);
+      float m_run = -INFINITY;
+      uint64_t lsum = f2(0.f, 0.f);
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        if (!(ok = warp_wait(&bars->s_full[t], j & 1, abort_flag, p.status))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        uint32_t sr[128];
+        tmem_ld128_sync(lane_base + C::col_s(t), sr);
+        const bool masked = (j + 1) * kBN > tile_lim;
+        if (masked) {
+          const int lim = row_lim - j * kBN;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row max (raw score units): four independent chains of 3-input max, one per 32 columns
+        float mxc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int b0 = 32 * k;
+          float m = fmax3(__uint_as_float(sr[b0]), __uint_as_float(sr[b0 + 1]), __uint_as_float(sr[b0 + 2]));
+#pragma unroll
+          for (int i = 3; i < 31; i += 2) m = fmax3(m, __uint_as_float(sr[b0 + i]), __uint_as_float(sr[b0 + i + 1]));
+          mxc[k] = fmaxf(m, __uint_as_float(sr[b0 + 31]));
+        }
+        const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), mxc[3]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        // Rescale O only when the max grew by more than the threshold (warp-uniform decision).
+        const bool need = m_new > m_run + kRescaleThreshold;
+        if (j == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2(m_run - m_new) : 1.f;  // m_run = -inf only for empty rows
+          if (need) {
+            float l0, l1;
+            f2_split(lsum, l0, l1);
+            lsum = f2(l0 * alpha, l1 * alpha);
+            m_run = m_new;
+          }
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t orr[32];
-            tmem_ld32_sync(lane_base + kColO + ch * 32, orr);
+            tmem_ld32_sync(lane_base + C::col_o(t) + ch * 32, orr);
 #pragma unroll
             for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-            tmem_st32(lane_base + kColO + ch * 32, orr);
+            tmem_st32(lane_base + C::col_o(t) + ch * 32, orr);
           }
         }
-      }
-      {
-        uint32_t h0[32], h1[32];
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        const uint64_t negm = f2(-m_use, -m_use);
+        uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+        const uint32_t p_addr = lane_base + C::col_p(t);
+        if (masked) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          h0[i] = pk[i];
-          h1[i] = pk[32 + i];
+          for (int ch = 0; ch < 4; ++ch) exp_chunk<false, kFp16>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) exp_chunk<true, kFp16>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         }
-        tmem_st32(lane_base + kColP, h0);
-        tmem_st32(lane_base + kColP + 32, h1);
+        lsum = f2_add(lsum, f2_add(acc0, acc1));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
-      m_run = m_new;
-    }
-    if (ok) ok = warp_wait(&bars->o_done, (n_kv - 1) & 1, abort_flag, p.status);
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool store = qi < Lq;
-      const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
+      if (ok) ok = warp_wait(&bars->o_done[t], 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        float l0, l1;
+        f2_split(lsum, l0, l1);
+        const float l_run = l0 + l1;
+        const bool empty = (m_run == -INFINITY);
+        const float inv_l = empty ? 0.f : 1.f / l_run;
+        const bool store = qi < Lq;
+        const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t orr[32];
-        tmem_ld32_sync(lane_base + kColO + ch * 32, orr);
-        if (store) {
-          if constexpr (kOutF32) {
-            float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + ch * 32);
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orr[32];
+          tmem_ld32_sync(lane_base + C::col_o(t) + ch * 32, orr);
+          if (store) {
+            if constexpr (kOutF32) {
+              float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + ch * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              out[i] = make_float4(__uint_as_float(orr[4 * i]) * inv_l, __uint_as_float(orr[4 * i + 1]) * inv_l,
-                                   __uint_as_float(orr[4 * i + 2]) * inv_l, __uint_as_float(orr[4 * i + 3]) * inv_l);
-          } else {
-            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow + ch * 32);
+              for (int i = 0; i < 8; ++i)
+                out[i] = make_float4(__uint_as_float(orr[4 * i]) * inv_l, __uint_as_float(orr[4 * i + 1]) * inv_l,
+                                     __uint_as_float(orr[4 * i + 2]) * inv_l, __uint_as_float(orr[4 * i + 3]) * inv_l);
+            } else {
+              uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow + ch * 32);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float* f = reinterpret_cast<const float*>(orr + 8 * i);
-              out[i] = make_uint4(pack2<kFp16>(f[0] * inv_l, f[1] * inv_l), pack2<kFp16>(f[2] * inv_l, f[3] * inv_l),
-                                  pack2<kFp16>(f[4] * inv_l, f[5] * inv_l), pack2<kFp16>(f[6] * inv_l, f[7] * inv_l));
+              for (int i = 0; i < 4; ++i) {
+                const float* f = reinterpret_cast<const float*>(orr + 8 * i);
+                out[i] = make_uint4(pack2<kFp16>(f[0] * inv_l, f[1] * inv_l), pack2<kFp16>(f[2] * inv_l, f[3] * inv_l),
+                                    pack2<kFp16>(f[4] * inv_l, f[5] * inv_l), pack2<kFp16>(f[6] * inv_l, f[7] * inv_l));
+              }
             }
           }
         }
-      }
-      if (store) {
-        const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
-                                            : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
-        p.lse[li] = l_run > 0.f ? (m_run + lg2(l_run)) * kLn2 : -INFINITY;
+        if (store) {
+          const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
+                                              : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
+          p.lse[li] = empty ? -INFINITY : (m_run + lg2(l_run)) * kLn2;
+        }
       }
     }
   }
@@ -439,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown -------------------------------------------------------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
   }
@@ -483,12 +590,17 @@ int launch_t(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
   const int smem = Cfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid;
+  cudaFuncAttributes fattr;
+  e = cudaFuncGetAttributes(&fattr, kern);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  if (fattr.numRegs != kLaunchRegs) return static_cast<int>(cudaErrorInvalidConfiguration);
+  long long blocks;
   if (a.cu_seqlens == nullptr)
-    grid = dim3((a.Nq + kBM - 1) / kBM, a.H, a.B);
+    blocks = static_cast<long long>(p.num_pairs) * a.B * a.H;
   else
-    grid = dim3(a.Nq / kBM + a.B, a.H, 1);
-  kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+    blocks = (static_cast<long long>(a.Nq) / (kTiles * kBM) + a.B) * a.H;
+  if (blocks > 0x7fffffffLL) return static_cast<int>(cudaErrorInvalidConfiguration);
+  kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(mq, mk, mv, p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -511,6 +623,7 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.H = a.H;
   p.Nq = a.Nq;
   p.Nk = a.Nk;
+  p.num_pairs = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal ? 1 : 0;
   if (a.D == 64) {

@@ -139,6 +139,16 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Register re-balancing between warpgroups (all four warps of a warpgroup execute the same one).
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -201,6 +211,14 @@ __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[12
       "tcgen05.wait::ld.sync.aligned;"
       : FA_R32(0), FA_R32(32), FA_R32(64), FA_R32(96)
       : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      FA_W8(0), FA_W8(8)
       : "memory");
 }
 
@@ -280,6 +298,65 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
   } else {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
   }
+}
+
+}  // namespace fa
+
+namespace fa {
+
+// ------------------------------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 arithmetic)
+
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of arguments x <= 0 on the FMA/ALU pipes instead of the MUFU unit.
+// x is split as x = n + f with n = round(x) (obtained by adding 1.5 * 2^23, which leaves n in the
+// low mantissa bits) and |f| <= 1/2; 2^f comes from a cubic fitted by a Remez exchange to minimise
+// the relative error on [-1/2, 1/2] (max 7.5e-5); 2^n is applied by adding n << 23 to the bits of
+// the result.  Arguments are clamped at -125 so the exponent field stays normal.
+__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float a, b;
+  f2_split(x, a, b);
+  a = fmaxf(a, -125.f);
+  b = fmaxf(b, -125.f);
+  const uint64_t xc = f2(a, b);
+  const uint64_t t = f2_add(xc, f2(kRound, kRound));
+  const uint64_t n = f2_add(t, f2(-kRound, -kRound));
+  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(fr, f2(kC3, kC3), f2(kC2, kC2));
+  p = f2_fma(p, fr, f2(kC1, kC1));
+  p = f2_fma(p, fr, f2(kC0, kC0));
+  float ta, tb, pa, pb;
+  f2_split(t, ta, tb);
+  f2_split(p, pa, pb);
+  const float ra = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+  const float rb = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
+  return f2(ra, rb);
 }
 
 }  // namespace fa

@@ -140,7 +140,8 @@ def test_causal_row_zero_is_first_value_row():
                           scale=0.125, out_dtype=torch.float32)
     vf, qf, kf = to_f64(v, "bf16"), to_f64(q, "bf16"), to_f64(k, "bf16")
     on = o.cpu().numpy()
-    assert np.array_equal(on[:, 0], vf[:, 0])  # a single visible key: O_0 = V_0 exactly
+    # a single visible key: O_0 = V_0 up to fp32 rounding of the one weight (exact in the oracle)
+    np.testing.assert_allclose(on[:, 0], vf[:, 0], rtol=1e-6, atol=1e-7)
     exp = 0.125 * np.einsum("bhd,bhd->bh", qf[:, 0], kf[:, 0])
     assert np.max(np.abs(lse.cpu().numpy()[:, :, 0] - exp)) <= 1e-3
 
