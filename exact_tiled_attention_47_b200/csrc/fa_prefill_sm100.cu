@@ -59,22 +59,40 @@ constexpr int kSoftmaxRegs = 216;
 constexpr int kControlRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kEmuEvery = 8;  // of every kEmuEvery column pairs ...
-#ifndef FA_EMU_PAIRS
-#define FA_EMU_PAIRS 3
+// ... this many take the polynomial exp2 (the MUFU unit is the tighter limit at D = 64, where the
+// MMA work per score is half that of D = 128)
+template <int D>
+constexpr int emu_pairs() {
+#ifdef FA_EMU_PAIRS
+  return FA_EMU_PAIRS;
+#else
+  return D == 64 ? 3 : 2;
 #endif
-constexpr int kEmuPairs = FA_EMU_PAIRS;  // ... this many take the polynomial exp2
+}
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kTileBytes = kBM * D * 2;
-  static constexpr int kKStages = (D == 64) ? 4 : 2;
-  static constexpr int kVStages = (D == 64) ? 4 : 2;
+#ifndef FA_KSTAGES_128
+#define FA_KSTAGES_128 2
+#endif
+#ifndef FA_VSTAGES_128
+#define FA_VSTAGES_128 2
+#endif
+  static constexpr int kKStages = (D == 64) ? 4 : FA_KSTAGES_128;
+  static constexpr int kVStages = (D == 64) ? 4 : FA_VSTAGES_128;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTiles * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
+  // With P in its own TMEM columns (D = 64) the next S of a tile is issued as soon as the softmax
+  // has read the current one; with P aliased into S (D = 128) it must follow the P*V product.
+#ifndef FA_FORCE_LATE_S
+#define FA_FORCE_LATE_S 0
+#endif
+  static constexpr bool kEarlyS = (D == 64) && !FA_FORCE_LATE_S;
   __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
   __device__ static constexpr uint32_t col_o(int t) { return t ? ((D == 64) ? 320u : 384u) : 256u; }
   __device__ static constexpr uint32_t col_p(int t) {
@@ -85,7 +103,7 @@ struct Cfg {
 struct Bars {
   uint64_t q_full[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -173,10 +191,10 @@ __device__ void write_empty_row(const FwdParams& p, int b, int h, int q_row0, in
 }
 
 // P for 32 score columns (chunk ch of the row): x = s * scale * log2(e) - m, p = 2^x (on the MUFU
-// unit, or -- for kEmuPairs of every kEmuEvery column pairs when kMixed -- by the FMA-pipe
+// unit, or -- for kEmu of every kEmuEvery column pairs when kMixed -- by the FMA-pipe
 // polynomial), row-sum accumulation in two packed fp32 chains, conversion to the input type and a
-// 16-column TMEM store (two 16-bit values per column).
-template <bool kMixed, bool kFp16>
+// 16-column TMEM store (two 16-bit values per 32-bit column, the layout the P*V MMA reads).
+template <bool kMixed, bool kFp16, int kEmu>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[128], int ch, uint64_t sl2x2, uint64_t negm,
                                           uint64_t& acc0, uint64_t& acc1, uint32_t p_addr) {
   uint32_t pk[16];
@@ -185,7 +203,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[128], int ch, uin
     const int c = ch * 32 + 2 * i;
     const uint64_t x = f2_fma(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
     uint64_t pe;
-    if (kMixed && (i % kEmuEvery) < kEmuPairs) {
+    if (kMixed && (i % kEmuEvery) < kEmu) {
       pe = exp2_poly_pair(x);
     } else {
       float x0, x1;
@@ -216,9 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- work unit: (b, h, pair of Q tiles) -----------------------------------------------------
   int b, h, pair;
   if (p.cu == nullptr) {
-    const int bh_count = p.B * p.H;
-    const int bh = blockIdx.x % bh_count;
-    pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x / bh_count);  // longest (causal) first
+    // all pairs of one (b, h) are consecutive, so they run together and share its K/V in L2;
+    // within a head the pair with the most key blocks (causal) goes first
+    const int bh = static_cast<int>(blockIdx.x / p.num_pairs);
+    pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x % p.num_pairs);
     b = bh / p.H;
     h = bh % p.H;
   } else {
@@ -274,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_free[t], 4);
       mbar_init(&bars->p_full[t], 4);
       mbar_init(&bars->o_done[t], 1);
     }
@@ -385,36 +405,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (n_kv[t] > 0) issue_s(t, 0);
         mma_commit(&bars->k_empty[0]);
       }
-      for (int j = 0; ok && j < n_max; ++j) {
-        const int vs = j % C::kVStages;
-        if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
-        const bool next = j + 1 < n_max;
-        bool k_next_ready = false;
-        for (int t = 0; t < kTiles; ++t) {
-          if (j >= n_kv[t]) continue;
-          if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          issue_pv(t, j);
-          if (j + 1 < n_kv[t]) {
-            if (!k_next_ready) {
-              const int ks = (j + 1) % C::kKStages;
-              if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
-              tc_fence_after();
-              k_next_ready = true;
-            }
-            issue_s(t, j + 1);
-          } else {
-            mma_commit(&bars->o_done[t]);
-          }
-        }
-        if (!ok) break;
-        mma_commit(&bars->v_empty[vs]);
-        if (next) {
-          if (!k_next_ready) {  // no tile needed K(j+1): still hand the stage back in order
+      if constexpr (C::kEarlyS) {
+        // S_t(j+1) as soon as softmax t has read S_t(j); then the P*V products of block j.
+        for (int j = 0; ok && j < n_max; ++j) {
+          if (j + 1 < n_max) {
             const int ks = (j + 1) % C::kKStages;
             if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
+            for (int t = 0; t < kTiles; ++t) {
+              if (j + 1 >= n_kv[t]) continue;
+              if (!(ok = mbar_wait(&bars->s_free[t], j & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              issue_s(t, j + 1);
+            }
+            if (!ok) break;
+            mma_commit(&bars->k_empty[ks]);
           }
-          mma_commit(&bars->k_empty[(j + 1) % C::kKStages]);
+          const int vs = j % C::kVStages;
+          if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
+          for (int t = 0; t < kTiles; ++t) {
+            if (j >= n_kv[t]) continue;
+            if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(t, j);
+            mma_commit(&bars->o_done[t]);
+          }
+          if (!ok) break;
+          mma_commit(&bars->v_empty[vs]);
+        }
+      } else {
+        // P_t aliases S_t: S_t(j+1) follows PV_t(j); the commit of S_t(j+1) also covers PV_t(j).
+        for (int j = 0; ok && j < n_max; ++j) {
+          const int vs = j % C::kVStages;
+          if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
+          const bool next = j + 1 < n_max;
+          bool k_next_ready = false;
+          for (int t = 0; t < kTiles; ++t) {
+            if (j >= n_kv[t]) continue;
+            if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(t, j);
+            if (j + 1 < n_kv[t]) {
+              if (!k_next_ready) {
+                const int ks = (j + 1) % C::kKStages;
+                if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+                k_next_ready = true;
+              }
+              issue_s(t, j + 1);
+            } else {
+              mma_commit(&bars->o_done[t]);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars->v_empty[vs]);
+          if (next) {
+            if (!k_next_ready) {  // no tile needed K(j+1): still hand the stage back in order
+              const int ks = (j + 1) % C::kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
+            }
+            mma_commit(&bars->k_empty[(j + 1) % C::kKStages]);
+          }
         }
       }
       // no tensor-core work may still be in flight when TMEM and shared memory are released
@@ -445,6 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         uint32_t sr[128];
         tmem_ld128_sync(lane_base + C::col_s(t), sr);
+        if constexpr (C::kEarlyS) {  // S_t may now be overwritten by the next block's scores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->s_free[t]);
+        }
         const bool masked = (j + 1) * kBN > tile_lim;
         if (masked) {
           const int lim = row_lim - j * kBN;
@@ -464,18 +519,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), mxc[3]);
         const float m_new = fmaxf(m_run, mx * sl2);
-        // Rescale O only when the max grew by more than the threshold (warp-uniform decision).
+        // Rescale O only when the max grew by more than the threshold (warp-uniform decision); with
+        // early S the multiplication of O waits below until P_t(j-1) V has landed in O.
         const bool need = m_new > m_run + kRescaleThreshold;
+        float alpha = 1.f;
+        bool rescale = false;
         if (j == 0) {
           m_run = m_new;
         } else if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m_run - m_new) : 1.f;  // m_run = -inf only for empty rows
+          rescale = true;
           if (need) {
+            alpha = ex2(m_run - m_new);  // m_run = -inf only for rows without any key
             float l0, l1;
             f2_split(lsum, l0, l1);
             lsum = f2(l0 * alpha, l1 * alpha);
             m_run = m_new;
           }
+        }
+        if constexpr (C::kEarlyS) {
+          // P_t(j-1) V must have landed before P_t is overwritten or O_t rescaled
+          if (j > 0 && !(ok = warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+        }
+        if (rescale) {
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t orr[32];
@@ -491,10 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t p_addr = lane_base + C::col_p(t);
         if (masked) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) exp_chunk<false, kFp16>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
+          for (int ch = 0; ch < 4; ++ch) exp_chunk<false, kFp16, 0>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         } else {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) exp_chunk<true, kFp16>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
+          for (int ch = 0; ch < 4; ++ch) exp_chunk<true, kFp16, emu_pairs<D>()>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         }
         lsum = f2_add(lsum, f2_add(acc0, acc1));
         tmem_wait_st();
@@ -502,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
-      if (ok) ok = warp_wait(&bars->o_done[t], 0, abort_flag, p.status);
+      // the last P_t V product (o_done is committed once per block with early S, once in total otherwise)
+      if (ok) ok = warp_wait(&bars->o_done[t], C::kEarlyS ? ((n - 1) & 1) : 0, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
         float l0, l1;
