@@ -66,7 +66,7 @@ constexpr int emu_pairs() {
 #ifdef FA_EMU_PAIRS
   return FA_EMU_PAIRS;
 #else
-  return D == 64 ? 3 : 2;
+  return D == 64 ? 1 : 1;
 #endif
 }
 
@@ -194,28 +194,56 @@ __device__ void write_empty_row(const FwdParams& p, int b, int h, int q_row0, in
 // unit, or -- for kEmu of every kEmuEvery column pairs when kMixed -- by the FMA-pipe
 // polynomial), row-sum accumulation in two packed fp32 chains, conversion to the input type and a
 // 16-column TMEM store (two 16-bit values per 32-bit column, the layout the P*V MMA reads).
+#ifndef FA_PACKED_MUFU
+#define FA_PACKED_MUFU 1
+#endif
+template <bool kMixed, bool kFp16, int kEmu>
+__device__ __forceinline__ void exp_chunk_regs(const uint32_t (&sr)[128], int ch, uint64_t sl2x2, uint64_t negm,
+                                               uint64_t& acc0, uint64_t& acc1, uint32_t (&pk)[16]) {
+#if !FA_PACKED_MUFU
+  float sl2, nm, u;
+  f2_split(sl2x2, sl2, u);
+  f2_split(negm, nm, u);
+  float sa = 0.f, sb = 0.f;
+#endif
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = ch * 32 + 2 * i;
+    float p0, p1;
+    if (kMixed && (i % kEmuEvery) < kEmu) {
+      const uint64_t x = f2_fma(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
+      const uint64_t pe = exp2_poly_pair(x);
+      if (i & 1) acc1 = f2_add(acc1, pe);
+      else acc0 = f2_add(acc0, pe);
+      f2_split(pe, p0, p1);
+    } else {
+#if FA_PACKED_MUFU
+      const uint64_t x = f2_fma(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
+      float x0, x1;
+      f2_split(x, x0, x1);
+      const uint64_t pe = f2(ex2(x0), ex2(x1));
+      if (i & 1) acc1 = f2_add(acc1, pe);
+      else acc0 = f2_add(acc0, pe);
+      f2_split(pe, p0, p1);
+#else
+      p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, nm));
+      p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, nm));
+      sa += p0;
+      sb += p1;
+#endif
+    }
+    pk[i] = pack2<kFp16>(p0, p1);
+  }
+#if !FA_PACKED_MUFU
+  acc0 = f2_add(acc0, f2(sa, sb));
+#endif
+}
+
 template <bool kMixed, bool kFp16, int kEmu>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[128], int ch, uint64_t sl2x2, uint64_t negm,
                                           uint64_t& acc0, uint64_t& acc1, uint32_t p_addr) {
   uint32_t pk[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int c = ch * 32 + 2 * i;
-    const uint64_t x = f2_fma(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
-    uint64_t pe;
-    if (kMixed && (i % kEmuEvery) < kEmu) {
-      pe = exp2_poly_pair(x);
-    } else {
-      float x0, x1;
-      f2_split(x, x0, x1);
-      pe = f2(ex2(x0), ex2(x1));
-    }
-    if (i & 1) acc1 = f2_add(acc1, pe);
-    else acc0 = f2_add(acc0, pe);
-    float p0, p1;
-    f2_split(pe, p0, p1);
-    pk[i] = pack2<kFp16>(p0, p1);
-  }
+  exp_chunk_regs<kMixed, kFp16, kEmu>(sr, ch, sl2x2, negm, acc0, acc1, pk);
   tmem_st16(p_addr + ch * 16, pk);
 }
 
@@ -268,20 +296,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int m0 = pair * (kTiles * kBM);
   const int diag = Lk - Lq;  // bottom-right causal alignment
-  int n_kv[kTiles];
-#pragma unroll
-  for (int t = 0; t < kTiles; ++t) {
+  // key blocks each tile needs (0: the tile is past the end, or no row of it sees a key)
+  auto blocks_of = [&](int t) {
     const int first = m0 + t * kBM;
     int kv_end = Lk;
     if (p.causal) kv_end = min(Lk, first + kBM + diag);
-    n_kv[t] = (first < Lq && kv_end > 0) ? (kv_end + kBN - 1) / kBN : 0;
-  }
-  const int n_max = max(n_kv[0], n_kv[1]);
+    return (first < Lq && kv_end > 0) ? (kv_end + kBN - 1) / kBN : 0;
+  };
+  const int n_kv0 = blocks_of(0), n_kv1 = blocks_of(1);
+  auto n_kv = [&](int t) { return t ? n_kv1 : n_kv0; };
+  const int n_max = max(n_kv0, n_kv1);
 
   // softmax warps of tiles without any visible key write O = 0, LSE = -inf directly
   if (warp < 8) {
     const int t = warp >> 2;
-    if (n_kv[t] == 0) {
+    if (n_kv(t) == 0) {
       const int qi = m0 + t * kBM + (warp & 3) * 32 + lane;
       if (qi < Lq) write_empty_row<D, kOutF32>(p, b, h, q_row0, qi);
     }
@@ -333,13 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmap_v);
       const uint64_t keep = l2_policy_evict_last();
       for (int t = 0; t < kTiles; ++t) {
-        if (n_kv[t] == 0) continue;
+        if (n_kv(t) == 0) continue;
         mbar_arrive_expect_tx(&bars->q_full[t], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d(&tmap_q, &bars->q_full[t], sQ(t) + pn * kPanelBytes, pn * 64, h, q_row0 + m0 + t * kBM);
       }
-      int last_k[4] = {-1, -1, -1, -1}, last_v[4] = {-1, -1, -1, -1};
+      int k_issued = 0, v_issued = 0;  // blocks whose K / V copies were started
       bool ok = true;
       for (int j = 0; j < n_max; ++j) {
         const int ks = j % C::kKStages, vs = j % C::kVStages;
@@ -348,21 +377,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d_hint(&tmap_k, &bars->k_full[ks], sK(ks) + pn * kPanelBytes, pn * 64, h, k_row0 + j * kBN, keep);
-        last_k[ks] = j;
+        k_issued = j + 1;
         if (!(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVStages) & 1) ^ 1, abort_flag, p.status))) break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d_hint(&tmap_v, &bars->v_full[vs], sV(vs) + pn * kPanelBytes, pn * 64, h, k_row0 + j * kBN, keep);
-        last_v[vs] = j;
+        v_issued = j + 1;
       }
       if (!ok) {  // let every copy this thread started land before the CTA exits
         for (int t = 0; t < kTiles; ++t)
-          if (n_kv[t] > 0) drain_wait(&bars->q_full[t], 0);
-        for (int st = 0; st < C::kKStages; ++st)
-          if (last_k[st] >= 0) drain_wait(&bars->k_full[st], (last_k[st] / C::kKStages) & 1);
-        for (int st = 0; st < C::kVStages; ++st)
-          if (last_v[st] >= 0) drain_wait(&bars->v_full[st], (last_v[st] / C::kVStages) & 1);
+          if (n_kv(t) > 0) drain_wait(&bars->q_full[t], 0);
+        // the newest copy into each stage is the last one that can still be in flight
+        for (int j = max(0, k_issued - C::kKStages); j < k_issued; ++j)
+          drain_wait(&bars->k_full[j % C::kKStages], (j / C::kKStages) & 1);
+        for (int j = max(0, v_issued - C::kVStages); j < v_issued; ++j)
+          drain_wait(&bars->v_full[j % C::kVStages], (j / C::kVStages) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -397,12 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // prologue: S_t(0) for both tiles
       for (int t = 0; t < kTiles && ok; ++t)
-        if (n_kv[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, p.status);
+        if (n_kv(t) > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, p.status);
       if (ok) ok = mbar_wait(&bars->k_full[0], 0, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < kTiles; ++t)
-          if (n_kv[t] > 0) issue_s(t, 0);
+          if (n_kv(t) > 0) issue_s(t, 0);
         mma_commit(&bars->k_empty[0]);
       }
       if constexpr (C::kEarlyS) {
@@ -412,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ks = (j + 1) % C::kKStages;
             if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
             for (int t = 0; t < kTiles; ++t) {
-              if (j + 1 >= n_kv[t]) continue;
+              if (j + 1 >= n_kv(t)) continue;
               if (!(ok = mbar_wait(&bars->s_free[t], j & 1, abort_flag, p.status))) break;
               tc_fence_after();
               issue_s(t, j + 1);
@@ -423,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vs = j % C::kVStages;
           if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
           for (int t = 0; t < kTiles; ++t) {
-            if (j >= n_kv[t]) continue;
+            if (j >= n_kv(t)) continue;
             if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
             tc_fence_after();
             issue_pv(t, j);
@@ -440,11 +470,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool next = j + 1 < n_max;
           bool k_next_ready = false;
           for (int t = 0; t < kTiles; ++t) {
-            if (j >= n_kv[t]) continue;
+            if (j >= n_kv(t)) continue;
             if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
             tc_fence_after();
             issue_pv(t, j);
-            if (j + 1 < n_kv[t]) {
+            if (j + 1 < n_kv(t)) {
               if (!k_next_ready) {
                 const int ks = (j + 1) % C::kKStages;
                 if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
@@ -476,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_increase<kSoftmaxRegs>();
     // ================================ softmax / epilogue =========================================
     const int t = warp >> 2;
-    const int n = n_kv[t];
+    const int n = n_kv(t);
     if (n > 0) {
       const int quarter = warp & 3;
       const int r = quarter * 32 + lane;
@@ -536,8 +566,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_run = m_new;
           }
         }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        const uint64_t negm = f2(-m_use, -m_use);
+        uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+        const uint32_t p_addr = lane_base + C::col_p(t);
+        // First half of P into registers; with early S the previous P_t V product may still be
+        // reading the P_t columns, so only then wait for it (it normally finished long before).
+        uint32_t pk0[16], pk1[16];
+        if (masked) {
+          exp_chunk_regs<false, kFp16, 0>(sr, 0, sl2x2, negm, acc0, acc1, pk0);
+          exp_chunk_regs<false, kFp16, 0>(sr, 1, sl2x2, negm, acc0, acc1, pk1);
+        } else {
+          exp_chunk_regs<true, kFp16, emu_pairs<D>()>(sr, 0, sl2x2, negm, acc0, acc1, pk0);
+          exp_chunk_regs<true, kFp16, emu_pairs<D>()>(sr, 1, sl2x2, negm, acc0, acc1, pk1);
+        }
         if constexpr (C::kEarlyS) {
-          // P_t(j-1) V must have landed before P_t is overwritten or O_t rescaled
           if (j > 0 && !(ok = warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag, p.status))) break;
           tc_fence_after();
         }
@@ -551,16 +594,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(lane_base + C::col_o(t) + ch * 32, orr);
           }
         }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        const uint64_t negm = f2(-m_use, -m_use);
-        uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-        const uint32_t p_addr = lane_base + C::col_p(t);
+        tmem_st16(p_addr, pk0);
+        tmem_st16(p_addr + 16, pk1);
         if (masked) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) exp_chunk<false, kFp16, 0>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
+          for (int ch = 2; ch < 4; ++ch) exp_chunk<false, kFp16, 0>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         } else {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) exp_chunk<true, kFp16, emu_pairs<D>()>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
+          for (int ch = 2; ch < 4; ++ch) exp_chunk<true, kFp16, emu_pairs<D>()>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         }
         lsum = f2_add(lsum, f2_add(acc0, acc1));
         tmem_wait_st();
