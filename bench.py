@@ -50,6 +50,28 @@ def peaks():
         return dict(FALLBACK), "fallback"
 
 
+CSRC = os.path.join(ROOT, "exact_tiled_attention_47_b200", "csrc")
+TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def measured_traffic(key, scale=1.0):
+    """DRAM bytes per launch from the committed ncu summary, or None if the kernel changed since."""
+    import hashlib
+    try:
+        with open(TRAFFIC) as fh:
+            ent = json.load(fh)[key]
+        h = hashlib.sha256()
+        for f in ent["files"]:
+            with open(os.path.join(CSRC, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest()[:16] != ent["source_sha"]:
+            return None
+        b = ent.get("dram_bytes", ent.get("dram_bytes_per_batch_item"))
+        return float(b) * scale
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def prefill_flops(B, H, Nq, Nk, D, causal):
     f = 4.0 * B * H * Nq * Nk * D
     return f / 2 if causal else f
@@ -135,8 +157,28 @@ def to_dev(bits, dtype, device):
     return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
 
 
+def rank_seed(cfg_seed: int, rank: int) -> int:
+    """Each rank processes its own batch of the workload (independent problems, weak scaling)."""
+    return cfg_seed + 1000 * rank
+
+
+def max_over_ranks(ms: float, dist=None, device="cuda") -> float:
+    """The job's time is the slowest rank's (all ranks take the same collective steps)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, ms_per_step_max: float, world: int) -> float:
+    """Units of all ranks per second of the slowest rank."""
+    return units_per_step_per_rank * world / (ms_per_step_max * 1e-3)
+
+
 def timed(fn, steps, stream, dist=None):
-    """Time `steps` calls of fn on `stream` with CUDA events; returns (ms total, max over ranks)."""
+    """Time `steps` calls of fn on `stream` with CUDA events; returns the max over ranks (ms)."""
     import torch
     if dist is not None:
         dist.barrier()
@@ -148,11 +190,8 @@ def timed(fn, steps, stream, dist=None):
         fn()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist)
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
 
@@ -248,14 +287,15 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
     B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
     scale = cfg["scale"]
     stream = torch.cuda.current_stream(dev)
-    seed = cfg["seed"] + 1000 * rank  # each rank: its own batch of the same workload
+    seed = rank_seed(cfg["seed"], rank)
     q, k, v = si.dense_qkv(seed, B, N, N, H, D, dt)
     qd, kd, vd = (to_dev(t, dt, dev) for t in (q, k, v))
     od = torch.empty_like(qd)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    causal = bool(cfg.get("causal", False))
 
     def step():
-        st = fa.fa_fwd(qd, kd, vd, od, lse, B, H, N, N, D, scale, True, None, stream)
+        st = fa.fa_fwd(qd, kd, vd, od, lse, B, H, N, N, D, scale, causal, None, stream)
         if st:
             raise fa.FAError(st, "fa_fwd")
 
@@ -266,14 +306,15 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
         ms = timed(step, args.steps, stream, dist)
     if fa.fa_device_status(clear=True) != 0:
         raise RuntimeError("device status set during the timed prefill run")
-    flops_step = prefill_flops(B, H, N, N, D, True)
+    flops_step = prefill_flops(B, H, N, N, D, causal)
     ms_step = ms / args.steps
     tflops_rank = flops_step / (ms_step * 1e-3) / 1e12
-    value = tflops_rank * world
+    value = whole_job_rate(flops_step, ms_step, world) / 1e12
     peak_b, peak_s = pk["bf16_tflops"], pk["bf16_tflops_sustained"]
     roof = {"bound": "tensor", "achieved": tflops_rank, "peak": peak_b, "unit": "TFLOP/s",
-            "frac": tflops_rank / peak_b, "traffic": None,
-            "kernel": "fa_fwd_kernel<64,bf16,out bf16>",
+            "frac": tflops_rank / peak_b, "traffic": measured_traffic(args.workload),
+            "traffic_unit": "bytes per launch (ncu dram read+write)",
+            "kernel": f"fa_fwd_kernel<{D},bf16,out bf16>",
             "peak_kind": f"{pk_kind} bf16 burst", "frac_of_sustained": tflops_rank / peak_s,
             "algorithmic_flops_per_launch": flops_step}
 
@@ -321,6 +362,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="profiling runs: time only one of the two paths")
+    ap.add_argument("--workload", choices=["prefill_d64", "prefill_d128"], default=HEADLINE,
+                    help="prefill workload of the headline leg (default: the D=64 configuration)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="profiling runs: smaller decode batch than the workload's B=64")
     args = ap.parse_args()
@@ -347,7 +390,7 @@ def main():
     pk, pk_kind = peaks()
 
     # ---------------- prefill headline ----------------
-    cfg = si.CONFIGS[HEADLINE]
+    cfg = si.CONFIGS[args.workload]
     run_prefill = args.only in ("all", "prefill")
     run_decode = args.only in ("all", "decode") and not args.no_decode
     B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
@@ -366,7 +409,7 @@ def main():
         Bd, Hd, Nk, Dd, S = c["B"], c["H"], c["Nk"], c["D"], c["num_splits"]
         if args.decode_batch:
             Bd = args.decode_batch
-        dseed = c["seed"] + 1000 * rank
+        dseed = rank_seed(c["seed"], rank)
         qd_ = to_dev(si.batched(dseed, si.Q_ID, Bd, (1, Hd, Dd), "bf16"), "bf16", dev)
         kc = torch.empty((Bd, Nk, Hd, Dd), dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
@@ -398,7 +441,7 @@ def main():
                "config": {"workload": "decode", "B": Bd, "H": Hd, "Nk": Nk, "D": Dd, "num_splits": S,
                           "dtype": "bf16", "l2": f"K/V cache {kv_bytes / 1e9:.2f} GB vs 126 MB L2"},
                "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                            "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                            "frac": gbs / pk["hbm_gbs"], "traffic": measured_traffic("decode", Bd),
                             "peak_kind": f"{pk_kind} copy", "algorithmic_bytes_per_step": alg_bytes},
                "gpu_launches": 2 * dsteps}
         del qd_, kc, vc, o_, l_, ws
@@ -420,9 +463,10 @@ def main():
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": HEADLINE, "B": B, "H": H, "N": N, "D": D, "causal": True,
-                   "input_dtype": dt, "output_dtype": "bf16", "scale": scale,
-                   "l2": "inputs 192 MiB > 126 MB L2 (no flush needed)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "D": D,
+                   "causal": bool(cfg.get("causal", False)), "input_dtype": dt, "output_dtype": "bf16",
+                   "scale": scale,
+                   "l2": f"inputs {3 * B * N * H * D * 2 / 2**20:.0f} MiB > 126 MB L2 (no flush needed)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof, "clocks": clk.summary(), "e2e": e2e,
         "gpu_launches": args.steps if run_prefill else 0,
