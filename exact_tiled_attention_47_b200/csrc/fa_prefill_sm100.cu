@@ -43,7 +43,7 @@ constexpr int kBN = 128;  // keys per block
 constexpr int kTiles = 2;
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;  // owns TMEM; issues the MMAs of tile 0 (warp 10 those of tile 1)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBM * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr float kLog2e = 1.4426950408889634f;
@@ -86,7 +86,7 @@ struct Cfg {
   static constexpr int kKOff = kQOff + kTiles * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kSmemBytes = kBarOff + 384 + 1024;  // barriers + alignment slack
   // With P in its own TMEM columns (D = 64) the next S of a tile is issued as soon as the softmax
   // has read the current one; with P aliased into S (D = 128) it must follow the P*V product.
 #ifndef FA_FORCE_LATE_S
@@ -102,14 +102,15 @@ struct Cfg {
 
 struct Bars {
   uint64_t q_full[2];
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t k_full[4], v_full[4];
+  uint64_t k_empty[2][4], v_empty[2][4];  // per tile: its MMAs no longer read the stage
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
   int tile_b, tile_pair;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block too large");
+static_assert(sizeof(Bars) <= 384, "barrier block too large");
 
 struct FwdParams {
   void* o;
@@ -328,13 +329,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->k_empty[0][s], 1);
+      mbar_init(&bars->k_empty[1][s], 1);
     }
     for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->v_empty[0][s], 1);
+      mbar_init(&bars->v_empty[1][s], 1);
     }
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -372,13 +376,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int j = 0; j < n_max; ++j) {
         const int ks = j % C::kKStages, vs = j % C::kVStages;
-        if (!(ok = mbar_wait(&bars->k_empty[ks], ((j / C::kKStages) & 1) ^ 1, abort_flag, p.status))) break;
+        // the stage's previous block must no longer be read by any tile that used it
+        const int jk = j - C::kKStages, jv = j - C::kVStages;
+        for (int t = 0; t < kTiles && ok && jk >= 0; ++t)
+          if (jk < n_kv(t)) ok = mbar_wait(&bars->k_empty[t][ks], (jk / C::kKStages) & 1, abort_flag, p.status);
+        if (!ok) break;
         mbar_arrive_expect_tx(&bars->k_full[ks], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d_hint(&tmap_k, &bars->k_full[ks], sK(ks) + pn * kPanelBytes, pn * 64, h, k_row0 + j * kBN, keep);
         k_issued = j + 1;
-        if (!(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVStages) & 1) ^ 1, abort_flag, p.status))) break;
+        for (int t = 0; t < kTiles && ok && jv >= 0; ++t)
+          if (jv < n_kv(t)) ok = mbar_wait(&bars->v_empty[t][vs], (jv / C::kVStages) & 1, abort_flag, p.status);
+        if (!ok) break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
@@ -395,111 +405,102 @@ __global__ void __launch_bounds__(kThreads, 1)
           drain_wait(&bars->v_full[j % C::kVStages], (j / C::kVStages) & 1);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ================================ MMA issuer =================================================
-    if (lane == 0) {
-      constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_qk = instr_desc_f16(kBM, kBN, fmt, 0);
-      constexpr uint32_t idesc_pv = instr_desc_f16(kBM, D, fmt, 1);
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ================================ MMA issuers ================================================
+    // Early S (D = 64): one issuing thread per tile (warp 9 for tile 0, warp 10 for tile 1), so
+    // neither tile's S or P*V waits behind the other's; the tensor core runs both streams in arrival
+    // order.  Late S (D = 128, P aliased into S): one thread (warp 9) issues both tiles in the order
+    // PV0(j) S0(j+1) PV1(j) S1(j+1), which keeps each tile's S right behind its own P*V.
+    // A commit covers only the issuing thread's earlier MMAs.
+    constexpr int fmt = kFp16 ? 0 : 1;
+    constexpr uint32_t idesc_qk = instr_desc_f16(kBM, kBN, fmt, 0);
+    constexpr uint32_t idesc_pv = instr_desc_f16(kBM, D, fmt, 1);
+    auto issue_s = [&](int t, int j) {
+      const uint32_t sQa = smem_addr(sQ(t));
+      const uint32_t sKa = smem_addr(sK(j % C::kKStages));
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row;
+        // every 4 steps move to the next 64-column panel.  SBO = 8 rows * 128 B.
+        const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
+        mma_ss(tbase + C::col_s(t), smem_desc_sw128(sQa + off, 16, 1024), smem_desc_sw128(sKa + off, 16, 1024),
+               idesc_qk, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars->s_full[t]);
+      mma_commit(&bars->k_empty[t][j % C::kKStages]);
+    };
+    auto issue_pv = [&](int t, int j) {
+      const uint32_t sVa = smem_addr(sV(j % C::kVStages));
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        // V is N-major (head dim contiguous): 16 keys = two 8-row swizzle atoms = 2048 bytes;
+        // LBO = distance between the 64-column panels, SBO = 8 rows * 128 B.
+        mma_ts(tbase + C::col_o(t), tbase + C::col_p(t) + kk * 8,
+               smem_desc_sw128(sVa + kk * 2048, kPanelBytes, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&bars->v_empty[t][j % C::kVStages]);
+    };
+    auto wait_k = [&](int j) {
+      return mbar_wait(&bars->k_full[j % C::kKStages], (j / C::kKStages) & 1, abort_flag, p.status);
+    };
+    auto wait_v = [&](int j) {
+      return mbar_wait(&bars->v_full[j % C::kVStages], (j / C::kVStages) & 1, abort_flag, p.status);
+    };
+    if constexpr (C::kEarlyS) {
+      const int t = warp - kMmaWarp;
+      const int n = n_kv(t);
+      if (lane == 0 && n > 0) {
+        bool ok = mbar_wait(&bars->q_full[t], 0, abort_flag, p.status) && wait_k(0);
+        if (ok) {
+          tc_fence_after();
+          issue_s(t, 0);
+        }
+        for (int j = 0; ok && j < n; ++j) {
+          // S_t(j+1) as soon as softmax t has read S_t(j); then P_t(j) V_j.
+          if (j + 1 < n) {
+            if (!(ok = wait_k(j + 1) && mbar_wait(&bars->s_free[t], j & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_s(t, j + 1);
+          }
+          if (!(ok = wait_v(j) && mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          mma_commit(&bars->o_done[t]);
+        }
+        // no tensor-core work of this thread may still be in flight when TMEM and SMEM are released
+        mma_commit(&bars->drain[t]);
+        drain_wait(&bars->drain[t], 0);
+      }
+    } else if (warp == kMmaWarp && lane == 0) {
       bool ok = true;
-      auto issue_s = [&](int t, int j) {
-        const uint32_t sQa = smem_addr(sQ(t));
-        const uint32_t sKa = smem_addr(sK(j % C::kKStages));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row;
-          // every 4 steps move to the next 64-column panel.  SBO = 8 rows * 128 B.
-          const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_ss(tbase + C::col_s(t), smem_desc_sw128(sQa + off, 16, 1024), smem_desc_sw128(sKa + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->s_full[t]);
-      };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t sVa = smem_addr(sV(j % C::kVStages));
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // V is N-major (head dim contiguous): 16 keys = two 8-row swizzle atoms = 2048 bytes;
-          // LBO = distance between the 64-column panels, SBO = 8 rows * 128 B.
-          mma_ts(tbase + C::col_o(t), tbase + C::col_p(t) + kk * 8,
-                 smem_desc_sw128(sVa + kk * 2048, kPanelBytes, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      // prologue: S_t(0) for both tiles
       for (int t = 0; t < kTiles && ok; ++t)
         if (n_kv(t) > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, p.status);
-      if (ok) ok = mbar_wait(&bars->k_full[0], 0, abort_flag, p.status);
+      if (ok) ok = wait_k(0);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < kTiles; ++t)
           if (n_kv(t) > 0) issue_s(t, 0);
-        mma_commit(&bars->k_empty[0]);
       }
-      if constexpr (C::kEarlyS) {
-        // S_t(j+1) as soon as softmax t has read S_t(j); then the P*V products of block j.
-        for (int j = 0; ok && j < n_max; ++j) {
-          if (j + 1 < n_max) {
-            const int ks = (j + 1) % C::kKStages;
-            if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
-            for (int t = 0; t < kTiles; ++t) {
-              if (j + 1 >= n_kv(t)) continue;
-              if (!(ok = mbar_wait(&bars->s_free[t], j & 1, abort_flag, p.status))) break;
-              tc_fence_after();
-              issue_s(t, j + 1);
-            }
-            if (!ok) break;
-            mma_commit(&bars->k_empty[ks]);
-          }
-          const int vs = j % C::kVStages;
-          if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
-          for (int t = 0; t < kTiles; ++t) {
-            if (j >= n_kv(t)) continue;
-            if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+      for (int j = 0; ok && j < n_max; ++j) {
+        if (!(ok = wait_v(j))) break;
+        bool k_next_ready = false;
+        for (int t = 0; t < kTiles; ++t) {
+          if (j >= n_kv(t)) continue;
+          if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          if (j + 1 < n_kv(t)) {  // P_t aliases S_t: S_t(j+1) follows P_t(j) V_j
+            if (!k_next_ready && !(ok = wait_k(j + 1))) break;
+            k_next_ready = true;
             tc_fence_after();
-            issue_pv(t, j);
+            issue_s(t, j + 1);
+          } else {
             mma_commit(&bars->o_done[t]);
           }
-          if (!ok) break;
-          mma_commit(&bars->v_empty[vs]);
-        }
-      } else {
-        // P_t aliases S_t: S_t(j+1) follows PV_t(j); the commit of S_t(j+1) also covers PV_t(j).
-        for (int j = 0; ok && j < n_max; ++j) {
-          const int vs = j % C::kVStages;
-          if (!(ok = mbar_wait(&bars->v_full[vs], (j / C::kVStages) & 1, abort_flag, p.status))) break;
-          const bool next = j + 1 < n_max;
-          bool k_next_ready = false;
-          for (int t = 0; t < kTiles; ++t) {
-            if (j >= n_kv(t)) continue;
-            if (!(ok = mbar_wait(&bars->p_full[t], j & 1, abort_flag, p.status))) break;
-            tc_fence_after();
-            issue_pv(t, j);
-            if (j + 1 < n_kv(t)) {
-              if (!k_next_ready) {
-                const int ks = (j + 1) % C::kKStages;
-                if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              issue_s(t, j + 1);
-            } else {
-              mma_commit(&bars->o_done[t]);
-            }
-          }
-          if (!ok) break;
-          mma_commit(&bars->v_empty[vs]);
-          if (next) {
-            if (!k_next_ready) {  // no tile needed K(j+1): still hand the stage back in order
-              const int ks = (j + 1) % C::kKStages;
-              if (!(ok = mbar_wait(&bars->k_full[ks], ((j + 1) / C::kKStages) & 1, abort_flag, p.status))) break;
-            }
-            mma_commit(&bars->k_empty[(j + 1) % C::kKStages]);
-          }
         }
       }
-      // no tensor-core work may still be in flight when TMEM and shared memory are released
-      mma_commit(&bars->drain);
-      drain_wait(&bars->drain, 0);
+      mma_commit(&bars->drain[0]);
+      drain_wait(&bars->drain[0], 0);
     }
   }
   } else {
@@ -573,7 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // First half of P into registers; with early S the previous P_t V product may still be
         // reading the P_t columns, so only then wait for it (it normally finished long before).
         uint32_t pk0[16], pk1[16];
-        if (masked) {
+#ifndef FA_UNIFIED_EXP
+#define FA_UNIFIED_EXP 0
+#endif
+        if (masked && !FA_UNIFIED_EXP) {
           exp_chunk_regs<false, kFp16, 0>(sr, 0, sl2x2, negm, acc0, acc1, pk0);
           exp_chunk_regs<false, kFp16, 0>(sr, 1, sl2x2, negm, acc0, acc1, pk1);
         } else {
@@ -596,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(p_addr, pk0);
         tmem_st16(p_addr + 16, pk1);
-        if (masked) {
+        if (masked && !FA_UNIFIED_EXP) {
 #pragma unroll
           for (int ch = 2; ch < 4; ++ch) exp_chunk<false, kFp16, 0>(sr, ch, sl2x2, negm, acc0, acc1, p_addr);
         } else {
