@@ -14,6 +14,10 @@ batch item (same page, "常见错误排查", error 4).
 
 Readings where the pages are silent:
   * causal with Nq != Nk is bottom-right aligned: query i sees key j iff j <= i + (Nk - Nq);
+  * the prefix mask, which the same page names among the mask formats of other architectures
+    ("原因分析", item 1) without defining it, is the prefix-LM mask: causal, except that the first
+    ``prefix`` keys are visible to every query (query i sees key j iff j < prefix or
+    j <= i + (Nk - Nq)); prefix = 0 is the causal mask;
   * a row with no visible key gets O = 0 and LSE = -inf;
   * LSE is the natural log-sum-exp of the scaled, masked scores of a row.
 
@@ -25,7 +29,7 @@ from __future__ import annotations
 import numpy as np
 
 
-def _visible_mask(nq: int, nk: int, causal: bool, k_valid: int | None) -> np.ndarray:
+def _visible_mask(nq: int, nk: int, causal: bool, k_valid: int | None, prefix: int = 0) -> np.ndarray:
     """Boolean [nq, nk]: True where query i may attend to key j."""
     j = np.arange(nk)[None, :]
     vis = np.ones((nq, nk), dtype=bool)
@@ -33,24 +37,25 @@ def _visible_mask(nq: int, nk: int, causal: bool, k_valid: int | None) -> np.nda
         vis &= j < k_valid
     if causal:
         i = np.arange(nq)[:, None]
-        vis &= j <= i + (nk - nq)
+        vis &= (j <= i + (nk - nq)) | (j < prefix)
     return vis
 
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, causal: bool = False,
-                   k_valid: int | None = None):
+                   k_valid: int | None = None, prefix: int = 0):
     """O [Nq, Dv] and LSE [Nq] for one (batch, head).
 
     q: [Nq, D], k: [Nk, D], v: [Nk, Dv], all float64.  ``k_valid`` (optional) masks keys j >= k_valid
-    (key padding).  Step 1: S = scale * Q K^T.  Masked entries become -inf.  Step 2: row softmax with
-    the row max m subtracted (safe softmax), P = exp(S - m), l = sum_j P.  Step 3: O = P V / l.
+    (key padding); ``prefix`` (causal only) makes the first ``prefix`` keys visible to every query.
+    Step 1: S = scale * Q K^T.  Masked entries become -inf.  Step 2: row softmax with the row max m
+    subtracted (safe softmax), P = exp(S - m), l = sum_j P.  Step 3: O = P V / l.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     nq, nk = q.shape[0], k.shape[0]
     s = scale * (q @ k.T)
-    vis = _visible_mask(nq, nk, causal, k_valid)
+    vis = _visible_mask(nq, nk, causal, k_valid, prefix)
     s = np.where(vis, s, -np.inf)
     o = np.zeros((nq, v.shape[1]), dtype=np.float64)
     lse = np.full(nq, -np.inf, dtype=np.float64)
@@ -65,7 +70,7 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, ca
     return o, lse
 
 
-def attention_dense(q, k, v, scale: float, causal: bool = False):
+def attention_dense(q, k, v, scale: float, causal: bool = False, prefix: int = 0):
     """Dense layout: q [B,Nq,H,D], k/v [B,Nk,H,D] float64 -> O [B,Nq,H,Dv], LSE [B,H,Nq]."""
     B, Nq, H, _ = q.shape
     Dv = v.shape[3]
@@ -74,15 +79,16 @@ def attention_dense(q, k, v, scale: float, causal: bool = False):
     for b in range(B):
         for h in range(H):
             o[b, :, h, :], lse[b, h, :] = attention_head(q[b, :, h, :], k[b, :, h, :], v[b, :, h, :],
-                                                         scale, causal)
+                                                         scale, causal, prefix=prefix)
     return o, lse
 
 
-def attention_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False):
+def attention_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False, prefix: int = 0):
     """Packed varlen self-attention: q/k/v [total,H,D]; sequence b owns rows cu[b]:cu[b+1].
 
     Each query of sequence b attends to exactly the keys of sequence b (the packed form of the 2-D
-    key-padding mask).  Returns O [total,H,Dv] and LSE [H,total].
+    key-padding mask); with ``causal`` the prefix (same length for every sequence) is counted from the
+    sequence's first key.  Returns O [total,H,Dv] and LSE [H,total].
     """
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     total, H, _ = q.shape
@@ -94,7 +100,7 @@ def attention_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False):
             continue
         for h in range(H):
             o[s0:s1, h, :], lse[h, s0:s1] = attention_head(q[s0:s1, h, :], k[s0:s1, h, :],
-                                                           v[s0:s1, h, :], scale, causal)
+                                                           v[s0:s1, h, :], scale, causal, prefix=prefix)
     return o, lse
 
 
@@ -125,7 +131,7 @@ def padded_key_mask_attention(q, k, v, key_mask, scale: float):
 
 
 def attention_rows(q_head, k_head, v_head, rows, scale: float, causal: bool = False,
-                   k_valid: int | None = None):
+                   k_valid: int | None = None, prefix: int = 0):
     """O and LSE of selected query rows of one (batch, head), each row evaluated on its own.
 
     q_head [Nq,D]; ``rows`` are query indices.  Used to check full-size runs on sampled outputs.
@@ -139,8 +145,8 @@ def attention_rows(q_head, k_head, v_head, rows, scale: float, causal: bool = Fa
     lse = np.full(len(rows), -np.inf)
     for r, i in enumerate(rows):
         last = nk if k_valid is None else k_valid
-        if causal:
-            last = min(last, int(i) + (nk - nq) + 1)
+        if causal:  # visible keys form the prefix [0, last) of the row
+            last = min(last, max(prefix, int(i) + (nk - nq) + 1))
         if last <= 0:
             continue
         s = scale * (k_head[:last] @ q_head[i])

@@ -12,8 +12,12 @@ from __future__ import annotations
 import math
 
 
-def brute_attention_head(q, k, v, scale: float, causal: bool = False, k_valid=None):
-    """q: [Nq][D], k: [Nk][D], v: [Nk][Dv] nested sequences of floats -> (O rows, LSE list)."""
+def brute_attention_head(q, k, v, scale: float, causal: bool = False, k_valid=None, prefix: int = 0):
+    """q: [Nq][D], k: [Nk][D], v: [Nk][Dv] nested sequences of floats -> (O rows, LSE list).
+
+    With ``causal`` a key is visible when it is at or before the query's diagonal position or among
+    the first ``prefix`` keys (prefix-LM mask; prefix = 0 is plain causal).
+    """
     q = [[float(x) for x in row] for row in q]
     k = [[float(x) for x in row] for row in k]
     v = [[float(x) for x in row] for row in v]
@@ -22,7 +26,7 @@ def brute_attention_head(q, k, v, scale: float, causal: bool = False, k_valid=No
     out, lse = [], []
     for i in range(nq):
         visible = [j for j in range(nk)
-                   if j < kv_len and (not causal or j <= i + (nk - nq))]
+                   if j < kv_len and (not causal or j <= i + (nk - nq) or j < prefix)]
         if not visible:
             out.append([0.0] * dv)
             lse.append(-math.inf)

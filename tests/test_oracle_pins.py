@@ -17,7 +17,10 @@ wrong LSE base, a bad group merge) fails at least one of them:
     materialised definition;
   * padded + 2-D key mask against packed varlen (to rounding, on valid rows);
   * split-KV partials + combine against the materialised single-query result;
-  * safe softmax: huge scores stay finite ("小知识" note under "内存卡点").
+  * safe softmax: huge scores stay finite ("小知识" note under "内存卡点");
+  * the prefix-LM mask: the Q = 0 closed form with its visible-key count, the limits prefix = 0
+    (causal) and prefix >= Nk (no mask), invariance under permutations inside the prefix (the prefix
+    is bidirectional), brute force, the row sampler and the packed varlen form.
 """
 import json
 import math
@@ -306,3 +309,83 @@ def test_row_sampler_matches_full_head():
         ro, rl = oracle.attention_rows(q, k, v, rows, 0.5, causal)
         np.testing.assert_allclose(ro, o[rows], rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(rl, lse[rows], rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# prefix-LM mask (causal with a bidirectional prefix of keys)
+
+
+@pytest.mark.parametrize("nq,nk,prefix", [(37, 37, 5), (20, 33, 9), (33, 20, 4), (16, 16, 40)])
+def test_prefix_zero_query_closed_form(nq, nk, prefix):
+    # Q = 0: every visible key has the same score, so O_i is the mean of the visible V rows and
+    # LSE_i = ln(#visible) with #visible = min(Nk, max(prefix, i + 1 + Nk - Nq)) (0 -> O = 0, -inf)
+    d = 8
+    q = np.zeros((nq, d))
+    k, v = rnd((nk, d), 101), rnd((nk, d), 102)
+    o, lse = oracle.attention_head(q, k, v, scale=0.3, causal=True, prefix=prefix)
+    for i in range(nq):
+        vis = min(nk, max(prefix, i + 1 + nk - nq))
+        if vis <= 0:
+            assert np.all(o[i] == 0) and lse[i] == -math.inf
+            continue
+        np.testing.assert_allclose(o[i], v[:vis].mean(axis=0), rtol=RTOL, atol=1e-14)
+        assert abs(lse[i] - math.log(vis)) < 1e-13
+
+
+def test_prefix_limits_are_causal_and_full():
+    nq, nk, d = 23, 23, 8
+    q, k, v = rnd((nq, d), 103), rnd((nk, d), 104), rnd((nk, d), 105)
+    oc, lc = oracle.attention_head(q, k, v, 0.25, causal=True)
+    o0, l0 = oracle.attention_head(q, k, v, 0.25, causal=True, prefix=0)
+    np.testing.assert_array_equal(o0, oc)
+    np.testing.assert_array_equal(l0, lc)
+    of, lf = oracle.attention_head(q, k, v, 0.25, causal=False)
+    on, ln = oracle.attention_head(q, k, v, 0.25, causal=True, prefix=nk)
+    np.testing.assert_array_equal(on, of)
+    np.testing.assert_array_equal(ln, lf)
+
+
+def test_prefix_keys_are_bidirectional():
+    # permuting keys (jointly with their values) inside the prefix leaves every row unchanged, which
+    # a causal treatment of the prefix would not
+    nq, nk, d, prefix = 19, 19, 8, 7
+    q, k, v = rnd((nq, d), 106), rnd((nk, d), 107), rnd((nk, d), 108)
+    perm = np.concatenate([np.random.default_rng(1).permutation(prefix), np.arange(prefix, nk)])
+    o1, l1 = oracle.attention_head(q, k, v, 0.2, causal=True, prefix=prefix)
+    o2, l2 = oracle.attention_head(q, k[perm], v[perm], 0.2, causal=True, prefix=prefix)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l2, l1, rtol=1e-13)
+    oc, _ = oracle.attention_head(q, k, v, 0.2, causal=True)
+    assert not np.allclose(o1[:prefix], oc[:prefix])  # the prefix rows do see later prefix keys
+
+
+@pytest.mark.parametrize("nq,nk,prefix", [(6, 6, 3), (5, 9, 2), (9, 5, 4), (16, 16, 1), (7, 13, 13)])
+def test_prefix_matches_brute_force(nq, nk, prefix):
+    d, dv = 6, 5
+    q, k, v = rnd((nq, d), 110 + nq), rnd((nk, d), 120 + nk), rnd((nk, dv), 130 + nk)
+    o, lse = oracle.attention_head(q, k, v, 0.3, True, prefix=prefix)
+    bo, bl = oracle.brute_attention_head(q.tolist(), k.tolist(), v.tolist(), 0.3, True, prefix=prefix)
+    bo, bl = np.array(bo), np.array(bl)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-14)
+    assert np.array_equal(np.isfinite(lse), np.isfinite(bl))
+    fin = np.isfinite(bl)
+    np.testing.assert_allclose(lse[fin], bl[fin], rtol=1e-13, atol=1e-14)
+
+
+def test_prefix_row_sampler_and_varlen():
+    nq, d, prefix = 70, 8, 25
+    q, k, v = rnd((nq, d), 131), rnd((nq, d), 132), rnd((nq, d), 133)
+    o, lse = oracle.attention_head(q, k, v, 0.5, True, prefix=prefix)
+    rows = [0, 1, 24, 25, 26, 69]
+    ro, rl = oracle.attention_rows(q, k, v, rows, 0.5, True, prefix=prefix)
+    np.testing.assert_allclose(ro, o[rows], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(rl, lse[rows], rtol=1e-13)
+    # packed varlen: the prefix counts from each sequence's first key
+    cu = [0, 30, 70]
+    qp, kp, vp = q[:, None, :], k[:, None, :], v[:, None, :]
+    vo, vl = oracle.attention_varlen(qp, kp, vp, cu, 0.5, causal=True, prefix=prefix)
+    for b in range(2):
+        s0, s1 = cu[b], cu[b + 1]
+        eo, el = oracle.attention_head(q[s0:s1], k[s0:s1], v[s0:s1], 0.5, True, prefix=prefix)
+        np.testing.assert_array_equal(vo[s0:s1, 0], eo)
+        np.testing.assert_array_equal(vl[0, s0:s1], el)
