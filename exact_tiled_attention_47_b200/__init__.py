@@ -18,7 +18,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
  FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT) = range(11)
 
 __all__ = [
-    "fa_fwd", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_status_string",
+    "fa_fwd", "fa_fwd_prefix", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
@@ -63,6 +63,19 @@ def fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu_seqlens=None, str
     return lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(H), int(Nq), int(Nk),
                       int(D), float(scale), int(bool(causal)), _ptr(cu_seqlens), _stream(stream),
                       int(in_dtype), int(o_dtype))
+
+
+def fa_fwd_prefix(q, k, v, o, lse, B, H, Nq, Nk, D, scale, prefix_len, cu_seqlens=None, stream=None,
+                  in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_fwd_prefix`` (causal with a bidirectional key prefix); returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    return lib.fa_fwd_prefix(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(H), int(Nq), int(Nk),
+                             int(D), float(scale), int(prefix_len), _ptr(cu_seqlens), _stream(stream),
+                             int(in_dtype), int(o_dtype))
 
 
 def fa_decode_workspace_bytes(B, H, D, num_splits) -> int:
@@ -129,8 +142,13 @@ def fa_abi_version() -> int:
 # allocating helpers (torch allocates; the library computes)
 
 
-def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None, stream=None):
-    """O, LSE for q [B,Nq,H,D], k/v [B,Nk,H,D] (dense) or packed [total,H,D] with cu_seqlens."""
+def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None, stream=None,
+              prefix_len=None):
+    """O, LSE for q [B,Nq,H,D], k/v [B,Nk,H,D] (dense) or packed [total,H,D] with cu_seqlens.
+
+    ``prefix_len`` (not None) selects the prefix mask (causal, with the first prefix_len keys visible
+    to every query); ``causal`` is then ignored.
+    """
     import torch
     D = q.shape[-1]
     if scale is None:
@@ -146,9 +164,12 @@ def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None
         B = cu_seqlens.numel() - 1
         lse = torch.empty((H, Nq), device=q.device, dtype=torch.float32)
     o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
-    st = fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu_seqlens, stream)
+    if prefix_len is None:
+        st = fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, cu_seqlens, stream)
+    else:
+        st = fa_fwd_prefix(q, k, v, o, lse, B, H, Nq, Nk, D, scale, prefix_len, cu_seqlens, stream)
     if st != FA_OK:
-        raise FAError(st, "fa_fwd")
+        raise FAError(st, "fa_fwd_prefix" if prefix_len is not None else "fa_fwd")
     return o, lse
 
 

@@ -84,15 +84,20 @@ const char* fa_status_string(int status) {
   }
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-           int D, float scale, int causal, const int* cu_seqlens, fa_stream_t stream, int in_dtype,
-           int o_dtype) {
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk, int D,
+             float scale, int causal, int prefix, const int* cu_seqlens, fa_stream_t stream, int in_dtype,
+             int o_dtype) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
   if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
   if (D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || H > 65535) return FA_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (prefix < 0) return FA_ERR_SHAPE;
   if (cu_seqlens) {
     if (Nq != Nk) return FA_ERR_SHAPE;  // self-attention: one packed extent for Q and K/V
     if (static_cast<int64_t>(Nq) / 128 + B > INT32_MAX) return FA_ERR_SHAPE;
@@ -123,6 +128,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   a.D = D;
   a.scale = scale;
   a.causal = causal != 0;
+  a.prefix = prefix;
   a.fp16 = in_dtype == FA_FP16;
   a.o_fp32 = o_dtype == FA_FP32;
   const int e = fa::launch_prefill(a, reinterpret_cast<cudaStream_t>(stream));
@@ -131,6 +137,23 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+           int D, float scale, int causal, const int* cu_seqlens, fa_stream_t stream, int in_dtype,
+           int o_dtype) {
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, D, scale, causal, 0, cu_seqlens, stream, in_dtype, o_dtype);
+}
+
+int fa_fwd_prefix(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                  int Nk, int D, float scale, int prefix_len, const int* cu_seqlens, fa_stream_t stream,
+                  int in_dtype, int o_dtype) {
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, D, scale, 1, prefix_len, cu_seqlens, stream, in_dtype,
+                  o_dtype);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits) {

@@ -18,6 +18,7 @@ struct PrefillArgs {
   int B, H, Nq, Nk, D;
   float scale;
   int causal;
+  int prefix;  // causal only: keys [0, prefix) are visible to every query (0 = plain causal)
   int fp16;    // input type: 1 = fp16, 0 = bf16
   int o_fp32;  // output type: 1 = fp32, 0 = input type
 };

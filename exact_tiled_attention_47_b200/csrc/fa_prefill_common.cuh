@@ -24,6 +24,7 @@ struct FwdParams {
   int num_units;  // dense: work units (groups of Q tiles) per (batch, head)
   float scale_log2;
   int causal;
+  int prefix;  // causal only: keys [0, prefix) of a sequence are visible to all its queries
 };
 
 // Bounded wait used only on the abort path: ignores the abort flag, has its own limit.

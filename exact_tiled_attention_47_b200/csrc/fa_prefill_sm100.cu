@@ -27,8 +27,8 @@
 // [384,448) P1 [448,512) (two 16-bit values per 32-bit column, the A operand of P*V read from TMEM);
 // D = 128: O0 [256,384) O1 [384,512) and P in shared memory (K-major, 128-byte swizzle, the A operand
 // of P*V read from shared memory), which leaves no room for more than one K stage.
-// Causal runs stop at the last key block the tile's last row can see; fully masked blocks are never
-// loaded or multiplied.  The pairs of one head run back to back (longest causal pair first) and
+// Causal runs (optionally with a prefix of keys every query sees, the prefix-LM mask) stop at the last
+// key block the tile's last row can see; fully masked blocks are never loaded or multiplied.  The pairs of one head run back to back (longest causal pair first) and
 // share its K/V in L2.
 #include <cudaTypedefs.h>
 
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto blocks_of = [&](int t) {
     const int first = m0 + t * kBM;
     int kv_end = Lk;
-    if (p.causal) kv_end = min(Lk, first + kBM + diag);
+    if (p.causal) kv_end = min(Lk, max(p.prefix, first + kBM + diag));
     return (first < Lq && kv_end > 0) ? (kv_end + kBN - 1) / kBN : 0;
   };
   const int n_kv0 = blocks_of(0), n_kv1 = blocks_of(1);
@@ -346,8 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
       const int tile_m0 = m0 + t * kBM;
       const int qi = tile_m0 + r;
-      const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;         // keys [0,row_lim) visible
-      const int tile_lim = p.causal ? min(Lk, tile_m0 + 1 + diag) : Lk;   // smallest row_lim of the tile
+      // keys [0, row_lim) are visible to this row; tile_lim is the smallest row_lim of the tile
+      const int row_lim = p.causal ? min(Lk, max(p.prefix, qi + 1 + diag)) : Lk;
+      const int tile_lim = p.causal ? min(Lk, max(p.prefix, tile_m0 + 1 + diag)) : Lk;
       const float sl2 = p.scale_log2;
       const uint64_t sl2x2 = f2(sl2, sl2);
       float m_run = -INFINITY;
@@ -523,6 +524,7 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.num_units = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal ? 1 : 0;
+  p.prefix = a.causal ? a.prefix : 0;
   if (a.D == 64) {
     if (a.fp16) return a.o_fp32 ? launch_t<64, true, true>(a, mq, mk, mv, p, stream) : launch_t<64, true, false>(a, mq, mk, mv, p, stream);
     return a.o_fp32 ? launch_t<64, false, true>(a, mq, mk, mv, p, stream) : launch_t<64, false, false>(a, mq, mk, mv, p, stream);

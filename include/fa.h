@@ -88,6 +88,23 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            const int* cu_seqlens, fa_stream_t stream, int in_dtype, int o_dtype);
 
 /*
+ * fa_fwd_prefix -- fa_fwd with the prefix mask: causal, except that the first prefix_len keys of each
+ * sequence are visible to every query of it (bidirectional attention over a prefix, causal after).
+ *
+ * Passage: the Hugging Face page, "原因分析" item 1, names the prefix mask (前缀掩码) next to the causal
+ * and bidirectional masks without defining it; the reading implemented is the prefix-LM mask:
+ * query i sees key j iff j < prefix_len or j <= i + (Nk_b - Nq_b).  prefix_len = 0 gives exactly
+ * fa_fwd(..., causal = 1, ...); prefix_len >= Nk gives the unmasked result.
+ *
+ * Arguments, layouts, ownership, limits and errors as fa_fwd (causal is implied), plus
+ * prefix_len >= 0 (negative -> FA_ERR_SHAPE).  In varlen mode the prefix is counted from the first
+ * key of every sequence.
+ */
+int fa_fwd_prefix(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int B, int H, int Nq, int Nk, int D, float scale, int prefix_len,
+                  const int* cu_seqlens, fa_stream_t stream, int in_dtype, int o_dtype);
+
+/*
  * fa_decode_workspace_bytes -- size of the scratch buffer fa_decode_splitkv needs:
  * num_splits * B * H * (D + 1) * 4 bytes (one fp32 partial output row and one fp32 partial LSE per
  * split), rounded up to 256 bytes.  Returns 0 for invalid arguments.

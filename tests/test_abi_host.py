@@ -104,6 +104,19 @@ def test_fwd_validation_codes(lib):
     assert _fwd(lib, cu=A + 2) == fa.FA_ERR_ALIGN
 
 
+def test_fwd_prefix_validation_codes(lib):
+    def pre(prefix, **kw):
+        a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, Nq=128, Nk=128, D=64, scale=0.125, cu=None)
+        a.update(kw)
+        return lib.fa_fwd_prefix(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"], a["Nk"],
+                                 a["D"], a["scale"], prefix, a["cu"], None, 0, 0)
+    assert pre(-1) == fa.FA_ERR_SHAPE
+    assert pre(10, q=None) == fa.FA_ERR_NULL
+    assert pre(10, D=96) == fa.FA_ERR_HEADDIM
+    assert pre(10, scale=0.0) == fa.FA_ERR_SHAPE
+    assert pre(10, o=A + 2) == fa.FA_ERR_ALIGN
+
+
 def _dec(lib, q=A, k=A, v=A, o=A, lse=A, B=2, H=2, Nk=64, D=128, scale=0.1, S=4, ws=A,
          wsb=1 << 20, in_dtype=0, o_dtype=0):
     return lib.fa_decode_splitkv(q, k, v, o, lse, B, H, Nk, D, scale, S, ws, wsb, None, in_dtype, o_dtype)
@@ -133,6 +146,7 @@ def test_device_status_null(lib):
 def test_no_device_is_reported(lib):
     # All arguments valid: the only failing check is the device one, and nothing is launched.
     assert _fwd(lib) == fa.FA_ERR_DEVICE
+    assert lib.fa_fwd_prefix(A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 10, None, None, 0, 0) == fa.FA_ERR_DEVICE
     assert _dec(lib) == fa.FA_ERR_DEVICE
     out = ctypes.c_int(0)
     assert lib.fa_device_status(ctypes.byref(out), 0) == fa.FA_ERR_DEVICE
