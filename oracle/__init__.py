@@ -7,20 +7,22 @@ library.  The two sides share only the seeded input generator, which holds no at
 
 Modules:
   attention  -- the materialised definition O = softmax(scale*Q*K^T + mask)*V with LSE, per (b, h);
-                dense, packed-varlen, row-sampled and single-query (decode) forms.
+                dense, packed-varlen, row-sampled and single-query (decode) forms, the latter also
+                with grouped KV heads and per-sequence cache lengths.
   online     -- the tiled algorithm in the order the pages give it (Q blocks outside, K/V blocks
                 inside, running max m and running sum l), and the pairwise merge of softmax
                 statistics of key groups, including the split-KV partial/combine form.
   brute      -- scalar pure-Python (math.fsum) evaluation for tiny inputs.
 """
 from .attention import (attention_head, attention_dense, attention_varlen, attention_rows,
-                        attention_decode, padded_key_mask_attention)
+                        attention_decode, attention_decode_gqa, padded_key_mask_attention)
 from .online import (tiled_online_attention, group_stats, merge_groups, softmax_by_groups,
                      split_kv_partials, combine_partials)
 from .brute import brute_attention_head
 
 __all__ = [
     "attention_head", "attention_dense", "attention_varlen", "attention_rows", "attention_decode",
+    "attention_decode_gqa",
     "padded_key_mask_attention", "tiled_online_attention", "group_stats", "merge_groups",
     "softmax_by_groups", "split_kv_partials", "combine_partials", "brute_attention_head",
 ]

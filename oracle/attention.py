@@ -165,3 +165,34 @@ def attention_decode(q, k_cache, v_cache, scale: float):
     verändert": prefill versus single-token decode differ only in the available parallelism).
     """
     return attention_dense(q, k_cache, v_cache, scale, causal=False)
+
+
+def attention_decode_gqa(q, k_cache, v_cache, scale: float, seqlens_k=None):
+    """Single-token decode with grouped KV heads and per-sequence cache lengths.
+
+    q [B,1,Hq,D]; k_cache/v_cache [B,Nk,Hkv,D] with Hq a multiple of Hkv; query head h reads KV head
+    h // (Hq // Hkv).  ``seqlens_k`` (optional, length B) gives the valid cache length of each batch
+    item: its query sees keys [0, seqlens_k[b]) (all Nk when omitted); a zero length gives O = 0 and
+    LSE = -inf.  Returns O [B,1,Hq,Dv] and LSE [B,Hq].
+
+    Reading: "Was FlashAttention bei Transformer-Inference verändert" asks whether a backend supports
+    the head dim, mask and cache layout and separates prefill from single-token decode, without
+    fixing a layout; grouped KV heads and per-sequence lengths are the plainest cache layout with
+    those two properties.
+    """
+    B, _, Hq, _ = q.shape
+    Nk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    o = np.zeros((B, 1, Hq, v_cache.shape[3]), dtype=np.float64)
+    lse = np.full((B, Hq), -np.inf, dtype=np.float64)
+    for b in range(B):
+        L = Nk if seqlens_k is None else int(seqlens_k[b])
+        if L <= 0:
+            continue
+        for h in range(Hq):
+            ob, lb = attention_head(q[b, :, h, :], k_cache[b, :L, h // G, :], v_cache[b, :L, h // G, :], scale)
+            o[b, :, h, :], lse[b, h] = ob, lb[0]
+    return o, lse
+

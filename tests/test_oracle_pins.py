@@ -20,7 +20,10 @@ wrong LSE base, a bad group merge) fails at least one of them:
   * safe softmax: huge scores stay finite ("小知识" note under "内存卡点");
   * the prefix-LM mask: the Q = 0 closed form with its visible-key count, the limits prefix = 0
     (causal) and prefix >= Nk (no mask), invariance under permutations inside the prefix (the prefix
-    is bidirectional), brute force, the row sampler and the packed varlen form.
+    is bidirectional), brute force, the row sampler and the packed varlen form;
+  * decode with grouped KV heads and per-sequence cache lengths: equal to the dense decode over KV
+    heads repeated G times, equal to decode over the truncated cache, the Q = 0 closed form, and
+    the split-KV combine with empty splits.
 """
 import json
 import math
@@ -389,3 +392,58 @@ def test_prefix_row_sampler_and_varlen():
         eo, el = oracle.attention_head(q[s0:s1], k[s0:s1], v[s0:s1], 0.5, True, prefix=prefix)
         np.testing.assert_array_equal(vo[s0:s1, 0], eo)
         np.testing.assert_array_equal(vl[0, s0:s1], el)
+
+
+# ---------------------------------------------------------------------------------------------
+# decode with grouped KV heads and per-sequence cache lengths
+
+
+def test_gqa_decode_equals_replicated_kv_heads():
+    # grouped heads are the dense decode over K/V heads repeated G times along the head axis
+    B, Nk, Hkv, G, D = 3, 50, 2, 4, 8
+    q = rnd((B, 1, Hkv * G, D), 140)
+    k, v = rnd((B, Nk, Hkv, D), 141), rnd((B, Nk, Hkv, D), 142)
+    o, lse = oracle.attention_decode_gqa(q, k, v, 0.3)
+    o_ref, lse_ref = oracle.attention_decode(q, np.repeat(k, G, axis=2), np.repeat(v, G, axis=2), 0.3)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, lse_ref[:, :, 0])
+
+
+def test_gqa_decode_lengths_truncate_the_cache():
+    B, Nk, Hkv, G, D = 4, 40, 3, 2, 8
+    q = rnd((B, 1, Hkv * G, D), 143)
+    k, v = rnd((B, Nk, Hkv, D), 144), rnd((B, Nk, Hkv, D), 145)
+    lens = [40, 1, 17, 0]
+    o, lse = oracle.attention_decode_gqa(q, k, v, 0.25, lens)
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert np.all(o[b] == 0) and np.all(lse[b] == -np.inf)
+            continue
+        ob, lb = oracle.attention_decode_gqa(q[b:b + 1], k[b:b + 1, :L], v[b:b + 1, :L], 0.25)
+        np.testing.assert_array_equal(o[b], ob[0])
+        np.testing.assert_array_equal(lse[b], lb[0])
+
+
+def test_gqa_decode_zero_query_closed_form():
+    # Q = 0: O is the mean of the first L value rows of the KV head, LSE = ln L
+    B, Nk, Hkv, G, D = 2, 30, 2, 3, 8
+    q = np.zeros((B, 1, Hkv * G, D))
+    k, v = rnd((B, Nk, Hkv, D), 146), rnd((B, Nk, Hkv, D), 147)
+    lens = [30, 7]
+    o, lse = oracle.attention_decode_gqa(q, k, v, 0.5, lens)
+    for b, L in enumerate(lens):
+        for h in range(Hkv * G):
+            np.testing.assert_allclose(o[b, 0, h], v[b, :L, h // G].mean(axis=0), rtol=RTOL, atol=1e-14)
+            assert abs(lse[b, h] - math.log(L)) < 1e-13
+
+
+def test_combine_of_empty_splits():
+    # splits past a short cache carry LSE = -inf and contribute nothing; the combine equals the
+    # materialised result
+    nk, splits, d = 5, 16, 8
+    q, k, v = rnd((d,), 148), rnd((nk, d), 149), rnd((nk, d), 150)
+    parts = oracle.split_kv_partials(q, k, v, 0.4, splits)
+    o, lse = oracle.combine_partials(*parts)
+    o_ref, lse_ref = oracle.attention_head(q[None, :], k, v, 0.4)
+    np.testing.assert_allclose(o, o_ref[0], rtol=1e-12, atol=1e-14)
+    assert abs(lse - lse_ref[0]) < 1e-12
