@@ -77,6 +77,14 @@ def prefill_flops(B, H, Nq, Nk, D, causal):
     return f / 2 if causal else f
 
 
+def prefix_flops(B, H, N, D, prefix):
+    """Algorithmic FLOPs of the prefix mask, counted per visible (query, key) pair: rows i < prefix
+    see prefix keys, rows i >= prefix see i + 1 keys (square self-attention)."""
+    p = min(max(prefix, 0), N)
+    pairs = p * p + (N * (N + 1) - p * (p + 1)) // 2
+    return 4.0 * B * H * D * pairs
+
+
 def causal_rows_flops(rows_lo, rows_hi, N, D):
     """Algorithmic FLOPs of query rows [lo, hi) of one causal head with Nq = Nk = N."""
     # row i sees i+1 keys: 4 * (i+1) * D
@@ -283,7 +291,7 @@ def run_reference(args):
 
 
 def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
-    """Time the headline prefill workload; returns (value, ms_step, roofline, e2e, clocks)."""
+    """Time the headline prefill workload; returns (value, ms_step, roofline, e2e, clocks, prefix)."""
     B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
     scale = cfg["scale"]
     stream = torch.cuda.current_stream(dev)
@@ -306,6 +314,31 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
         ms = timed(step, args.steps, stream, dist)
     if fa.fa_device_status(clear=True) != 0:
         raise RuntimeError("device status set during the timed prefill run")
+
+    # the same inputs under the prefix mask (a quarter of the keys visible to every query)
+    prefix = None
+    if causal and not args.no_prefix:
+        plen = N // 4
+
+        def pstep():
+            st = fa.fa_fwd_prefix(qd, kd, vd, od, lse, B, H, N, N, D, scale, plen, None, stream)
+            if st:
+                raise fa.FAError(st, "fa_fwd_prefix")
+
+        for _ in range(args.warmup):
+            pstep()
+        psteps = max(10, min(args.steps, 50))
+        ms_p = timed(pstep, psteps, stream, dist)
+        if fa.fa_device_status(clear=True) != 0:
+            raise RuntimeError("device status set during the timed prefix run")
+        pf = prefix_flops(B, H, N, D, plen)
+        ptf = pf / (ms_p / psteps * 1e-3) / 1e12
+        prefix = {"metric": "prefix-LM attention fwd TFLOPS", "value": whole_job_rate(pf, ms_p / psteps, world) / 1e12,
+                  "unit": "TFLOP/s", "ms_per_step": ms_p / psteps, "steps": psteps, "prefix_len": plen,
+                  "algorithmic_flops_per_launch": pf,
+                  "roofline": {"bound": "tensor", "achieved": ptf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                               "frac": ptf / pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst"},
+                  "gpu_launches": psteps}
     flops_step = prefill_flops(B, H, N, N, D, causal)
     ms_step = ms / args.steps
     tflops_rank = flops_step / (ms_step * 1e-3) / 1e12
@@ -347,7 +380,7 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
     del qd, kd, vd, od, lse
     torch.cuda.empty_cache()
 
-    return value, ms_step, roof, e2e, clk
+    return value, ms_step, roof, e2e, clk, prefix
 
 
 def main():
@@ -358,6 +391,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefix", action="store_true", help="skip the prefix-mask timing of the prefill inputs")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
@@ -397,10 +431,11 @@ def main():
     scale = cfg["scale"]
     stream = torch.cuda.current_stream(dev)
     value = ms_step = None
-    roof = e2e = None
+    roof = e2e = prefix = None
     clk = ClockSampler(local)
     if run_prefill:
-        value, ms_step, roof, e2e, clk = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch)
+        value, ms_step, roof, e2e, clk, prefix = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa,
+                                                             torch)
 
     # ---------------- decode (secondary metric) ----------------
     dec = None
@@ -447,6 +482,51 @@ def main():
         del qd_, kc, vc, o_, l_, ws
         torch.cuda.empty_cache()
 
+        # grouped KV heads with per-sequence cache lengths
+        g = si.CONFIGS["decode_gqa"]
+        Bg, Hq, Hkv, Nkg, Dg, Sg = g["B"], g["H"], g["Hkv"], g["Nk"], g["D"], g["num_splits"]
+        if args.decode_batch:
+            Bg = args.decode_batch
+        gseed = rank_seed(g["seed"], rank)
+        lens = si.varlen_lengths(g["seed"], Bg, g["len_lo"], g["len_hi"])
+        qg = to_dev(si.batched(gseed, si.Q_ID, Bg, (1, Hq, Dg), "bf16"), "bf16", dev)
+        kg = torch.empty((Bg, Nkg, Hkv, Dg), dtype=torch.bfloat16, device=dev)
+        vg = torch.empty_like(kg)
+        for b in range(Bg):
+            kg[b].copy_(to_dev(si.batch_item(gseed, si.K_ID, b, (Nkg, Hkv, Dg), "bf16"), "bf16", dev))
+            vg[b].copy_(to_dev(si.batch_item(gseed, si.V_ID, b, (Nkg, Hkv, Dg), "bf16"), "bf16", dev))
+        sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+        og = torch.empty_like(qg)
+        lg_ = torch.empty((Bg, Hq), dtype=torch.float32, device=dev)
+        wsbg = fa.fa_decode_workspace_bytes(Bg, Hq, Dg, Sg)
+        wsg = torch.empty(wsbg, dtype=torch.uint8, device=dev)
+
+        def gstep():
+            st = fa.fa_decode_splitkv_gqa(qg, kg, vg, og, lg_, Bg, Hq, Hkv, Nkg, Dg, g["scale"], Sg, sl, wsg, wsbg,
+                                          stream)
+            if st:
+                raise fa.FAError(st, "fa_decode_splitkv_gqa")
+
+        for _ in range(args.warmup):
+            gstep()
+        ms_g = timed(gstep, dsteps, stream, dist)
+        if fa.fa_device_status(clear=True) != 0:
+            raise RuntimeError("device status set during the timed grouped decode run")
+        kv_g = 2 * int(lens.sum()) * Hkv * Dg * 2  # valid K and V rows only
+        alg_g = kv_g + 2 * Bg * Hq * Dg * 2 + Bg * Hq * 4
+        gbs_g = alg_g / (ms_g / dsteps * 1e-3) / 1e9
+        dec["gqa"] = {"metric": "grouped decode HBM GB/s", "value": gbs_g * world, "unit": "GB/s",
+                      "ms_per_step": ms_g / dsteps, "steps": dsteps,
+                      "config": {"workload": "decode_gqa", "B": Bg, "Hq": Hq, "Hkv": Hkv, "Nk_capacity": Nkg,
+                                 "D": Dg, "num_splits": Sg, "lengths": f"U{{{g['len_lo']}..{g['len_hi']}}}",
+                                 "valid_kv_bytes": kv_g},
+                      "roofline": {"bound": "hbm", "achieved": gbs_g, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs_g / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy",
+                                   "algorithmic_bytes_per_step": alg_g},
+                      "gpu_launches": 2 * dsteps}
+        del qg, kg, vg, og, lg_, wsg, sl
+        torch.cuda.empty_cache()
+
     # ---------------- CPU baseline (oracle) ----------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and run_prefill:
@@ -470,7 +550,7 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof, "clocks": clk.summary(), "e2e": e2e,
         "gpu_launches": args.steps if run_prefill else 0,
-        "decode": dec, "cpu_baseline": cpu,
+        "decode": dec, "prefix": prefix, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     return 0

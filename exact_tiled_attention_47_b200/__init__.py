@@ -18,7 +18,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
  FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT) = range(11)
 
 __all__ = [
-    "fa_fwd", "fa_fwd_prefix", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_status_string",
+    "fa_fwd", "fa_fwd_prefix", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
@@ -80,6 +80,22 @@ def fa_fwd_prefix(q, k, v, o, lse, B, H, Nq, Nk, D, scale, prefix_len, cu_seqlen
 
 def fa_decode_workspace_bytes(B, H, D, num_splits) -> int:
     return int(load().fa_decode_workspace_bytes(int(B), int(H), int(D), int(num_splits)))
+
+
+def fa_decode_splitkv_gqa(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                          workspace, workspace_bytes=None, stream=None, in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_splitkv_gqa``; returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_decode_splitkv_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), int(B), int(Hq),
+                                     int(Hkv), int(Nk), int(D), float(scale), int(num_splits), _ptr(seqlens_k),
+                                     _ptr(workspace), int(workspace_bytes), _stream(stream), int(in_dtype),
+                                     int(o_dtype))
 
 
 def fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace,
@@ -174,11 +190,15 @@ def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None
 
 
 def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, workspace=None,
-           stream=None):
-    """O [B,1,H,D], LSE [B,H] for one query per (batch, head) over the cache [B,Nk,H,D]."""
+           stream=None, seqlens_k=None):
+    """O [B,1,Hq,D], LSE [B,Hq] for one query per (batch, head) over the cache [B,Nk,Hkv,D].
+
+    Hkv < Hq (a divisor of it) or ``seqlens_k`` (int32 [B] on the device) select the grouped /
+    ragged entry point ``fa_decode_splitkv_gqa``.
+    """
     import torch
     B, _, H, D = q.shape
-    Nk = k_cache.shape[1]
+    Nk, Hkv = k_cache.shape[1], k_cache.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     out_dtype = q.dtype if out_dtype is None else out_dtype
@@ -187,8 +207,12 @@ def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, works
         workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
     o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
     lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
-    st = fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace,
-                           workspace.numel() * workspace.element_size(), stream)
+    nb = workspace.numel() * workspace.element_size()
+    if Hkv == H and seqlens_k is None:
+        st = fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace, nb, stream)
+    else:
+        st = fa_decode_splitkv_gqa(q, k_cache, v_cache, o, lse, B, H, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                                   workspace, nb, stream)
     if st != FA_OK:
-        raise FAError(st, "fa_decode_splitkv")
+        raise FAError(st, "fa_decode_splitkv" if Hkv == H and seqlens_k is None else "fa_decode_splitkv_gqa")
     return o, lse

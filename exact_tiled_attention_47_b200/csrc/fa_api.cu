@@ -75,7 +75,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_HEADDIM: return "unsupported head dimension (must be 64 or 128)";
     case FA_ERR_SHAPE: return "invalid shape, split count or scale";
     case FA_ERR_ALIGN: return "a tensor pointer is misaligned (16 bytes; lse 4 bytes)";
-    case FA_ERR_CU_SEQLENS: return "cu_seqlens is not non-decreasing within the packed extent";
+    case FA_ERR_CU_SEQLENS: return "sequence lengths out of range (cu_seqlens must be non-decreasing within the packed extent, seqlens_k within [0, Nk])";
     case FA_ERR_WORKSPACE: return "decode workspace missing or too small";
     case FA_ERR_DEVICE: return "no usable sm_100 (B200) CUDA device";
     case FA_ERR_LAUNCH: return "CUDA launch or driver call failed";
@@ -163,14 +163,19 @@ size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits) {
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
-int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
-                      int H, int Nk, int D, float scale, int num_splits, void* workspace,
-                      size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype) {
+}  // extern "C"
+
+namespace {
+
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
+                int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k, void* workspace,
+                size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype) {
   if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_NULL;
   if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
   if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
   if (D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || Nk < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_SHAPE;
   if (num_splits < 1 || num_splits > 128) return FA_ERR_SHAPE;
   if (static_cast<int64_t>(B) * H > (static_cast<int64_t>(1) << 28)) return FA_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
@@ -178,6 +183,7 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, v
     return FA_ERR_ALIGN;
   if (!workspace || workspace_bytes < fa_decode_workspace_bytes(B, H, D, num_splits)) return FA_ERR_WORKSPACE;
   if (!fa::aligned(workspace, 16)) return FA_ERR_ALIGN;
+  if (seqlens_k && !fa::aligned(seqlens_k, 4)) return FA_ERR_ALIGN;
   int dev = -1;
   if (const int st = fa::check_device(&dev)) return st;
   int* status = fa::device_status_ptr();
@@ -200,12 +206,33 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, v
   a.scale = scale;
   a.fp16 = in_dtype == FA_FP16;
   a.o_fp32 = o_dtype == FA_FP32;
+  a.Hkv = Hkv;
+  a.seqlens_k = seqlens_k;
   const int e = fa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != 0) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
+                      int H, int Nk, int D, float scale, int num_splits, void* workspace,
+                      size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype) {
+  return decode_impl(q, k_cache, v_cache, o, lse, B, H, H, Nk, D, scale, num_splits, nullptr, workspace,
+                     workspace_bytes, stream, in_dtype, o_dtype);
+}
+
+int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k,
+                          void* workspace, size_t workspace_bytes, fa_stream_t stream, int in_dtype,
+                          int o_dtype) {
+  return decode_impl(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k, workspace,
+                     workspace_bytes, stream, in_dtype, o_dtype);
 }
 
 int fa_device_status(int* status_out, int clear) {

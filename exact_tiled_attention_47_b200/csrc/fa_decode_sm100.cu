@@ -5,14 +5,17 @@
 // cores with wide streaming loads rather than on the tensor cores ("Was FlashAttention bei
 // Transformer-Inference verändert": prefill and single-token decode expose different parallelism).
 //
-// Kernel 1 (split): CTA = (head, split, batch).  The split's keys are processed in chunks of
-//   kChunk: all scores of a chunk go to shared memory, then the chunk max updates the running max,
-//   the accumulator is rescaled and the value rows are accumulated with p = 2^(s - m).  The CTA
-//   writes the split's normalised partial output o_s and its natural-log LSE lse_s (fp32).
+// Kernel 1 (split): CTA = (group of G query heads sharing one KV head, split, batch).  The split's
+//   keys (of the batch item's valid cache length) are processed in chunks of kChunk: each K row
+//   slice is loaded once and dotted with the G queries, all scores of a chunk go to shared memory,
+//   then each head's chunk max updates its running max, its accumulator is rescaled and the value
+//   rows (again loaded once for the G heads) are accumulated with p = 2^(s - m).  The CTA writes
+//   each head's normalised partial output o_s and its natural-log LSE lse_s (fp32).  A split with
+//   no keys writes o_s = 0, lse_s = -inf.
 // Kernel 2 (combine): one warp per (batch, head) merges the splits: M = max_s lse_s,
 //   w_s = exp(lse_s - M), O = sum_s w_s o_s / sum_s w_s, LSE = M + ln sum_s w_s -- the pairwise
 //   merge of group statistics of "轻松读懂FlashAttention 上" ("Softmax求解重构") applied to all
-//   splits at once.
+//   splits at once; a query without any key (valid length 0) gets O = 0, LSE = -inf.
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 
@@ -21,6 +24,9 @@ namespace {
 
 constexpr int kDecThreads = 128;
 constexpr int kChunk = 256;
+// A split covers at least this many keys: shorter caches use fewer splits (the rest exit at once),
+// since a CTA's fixed costs (query load, reductions, partial writes) outweigh streaming a few keys.
+constexpr int kMinSplitKeys = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -32,7 +38,10 @@ struct DecParams {
   float* lse;
   float* ws_o;
   float* ws_lse;
-  int B, H, Nk, S;
+  const int* seqlens_k;  // nullable
+  int* status;
+  int B, H, Nk, S;  // H: query heads
+  int Hkv, group;   // KV heads; query heads per KV head (H = Hkv * group)
   float scale_log2;
 };
 
@@ -45,52 +54,73 @@ __device__ __forceinline__ void load8_stream(const void* ptr, float (&f)[8]) {
   f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
 
-template <bool kFp16, int D>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecParams p) {
+template <bool kFp16, int D, int G>
+__global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_kernel(const DecParams p) {
   using T = uint16_t;
   constexpr int LPK = D / 8;       // lanes sharing one key row (16-byte slice each)
   constexpr int KPW = 32 / LPK;    // keys per warp per step
   constexpr int KPB = KPW * 4;     // keys per CTA per step
-  constexpr int UNR = 4;           // independent row loads in flight per thread
+  constexpr int UNR = G >= 8 ? 2 : 4;  // independent row loads in flight per thread (registers)
 
-  const int h = blockIdx.x, s = blockIdx.y, b = blockIdx.z;
-  const int per = (p.Nk + p.S - 1) / p.S;
-  const int lo = min(p.Nk, s * per);
-  const int hi = min(p.Nk, lo + per);
+  const int s = blockIdx.y, b = blockIdx.z;
+  const int subs = p.group / G;  // CTAs per KV head
+  const int hk = blockIdx.x / subs;
+  const int hq0 = hk * p.group + (blockIdx.x % subs) * G;  // first of this CTA's G query heads
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = lane % LPK, kk = lane / LPK;
 
-  __shared__ float sc[kChunk];
-  __shared__ float red_m[4];
-  __shared__ float red_l[4];
-  __shared__ float red_acc[4][D];
+  int len = p.Nk;
+  if (p.seqlens_k != nullptr) {
+    len = __ldg(p.seqlens_k + b);
+    if (len < 0 || len > p.Nk) {  // reported, and the batch item is treated as having no keys
+      if (tid == 0 && s == 0 && blockIdx.x == 0) record_status(p.status, kStatusCuSeqlens);
+      len = 0;
+    }
+  }
+  const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
+  const int lo = min(len, s * per);
+  const int hi = min(len, lo + per);
 
-  const size_t bh = static_cast<size_t>(b) * p.H + h;
-  float* wo = p.ws_o + (bh * p.S + s) * D;
-  float* wl = p.ws_lse + bh * p.S + s;
-  if (lo >= hi) {  // a split past the end of the cache: empty partial
-    for (int d = tid; d < D; d += kDecThreads) wo[d] = 0.f;
-    if (tid == 0) *wl = -INFINITY;
+  __shared__ float sc[G][kChunk];
+  __shared__ float red_m[4][G];
+  __shared__ float red_l[4][G];
+  __shared__ float red_acc[4][G][D];
+
+  auto ws_o = [&](int g) { return p.ws_o + ((static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s) * D; };
+  auto ws_l = [&](int g) { return p.ws_lse + (static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s; };
+  if (lo >= hi) {  // a split past the end of the valid cache: empty partials
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      for (int d = tid; d < D; d += kDecThreads) ws_o(g)[d] = 0.f;
+      if (tid == 0) *ws_l(g) = -INFINITY;
+    }
     return;
   }
 
-  float qf[8];
-  load8_stream<kFp16>(static_cast<const T*>(p.q) + bh * D + c * 8, qf);
+  float qf[G][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) qf[e] *= p.scale_log2;  // scores come out in log2 units
-
-  const size_t rs = static_cast<size_t>(p.H) * D;  // elements between consecutive cache rows
-  const T* kb = static_cast<const T*>(p.k) + static_cast<size_t>(b) * p.Nk * rs + h * D + c * 8;
-  const T* vb = static_cast<const T*>(p.v) + static_cast<size_t>(b) * p.Nk * rs + h * D + c * 8;
-
-  float m_run = -INFINITY, l_part = 0.f;
-  float acc[8];
+  for (int g = 0; g < G; ++g) {
+    load8_stream<kFp16>(static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.H + hq0 + g) * D + c * 8, qf[g]);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;  // scores come out in log2 units
+  }
+
+  const size_t rs = static_cast<size_t>(p.Hkv) * D;  // elements between consecutive cache rows
+  const T* kb = static_cast<const T*>(p.k) + static_cast<size_t>(b) * p.Nk * rs + hk * D + c * 8;
+  const T* vb = static_cast<const T*>(p.v) + static_cast<size_t>(b) * p.Nk * rs + hk * D + c * 8;
+
+  float m_run[G], l_part[G], acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m_run[g] = -INFINITY;
+    l_part[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+  }
 
   for (int c0 = lo; c0 < hi; c0 += kChunk) {
     const int n = min(kChunk, hi - c0);
-    // scores of this chunk
+    // scores of this chunk: each K row slice is loaded once for the G queries
     for (int j0 = warp * KPW; j0 < n; j0 += UNR * KPB) {
       float kf[UNR][8];
 #pragma unroll
@@ -105,29 +135,39 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecPara
       }
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
-        float d = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(qf[e], kf[u][e], d);
-#pragma unroll
-        for (int o = LPK / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
         const int j = j0 + u * KPB + kk;
-        if (j < n && c == 0) sc[j] = d;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d = fmaf(qf[g][e], kf[u][e], d);
+#pragma unroll
+          for (int o = LPK / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+          if (j < n && c == 0) sc[g][j] = d;
+        }
       }
     }
     __syncthreads();
-    float mx = -INFINITY;
-    for (int j = tid; j < n; j += kDecThreads) mx = fmaxf(mx, sc[j]);
+    float m_new[G];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red_m[warp] = mx;
+    for (int g = 0; g < G; ++g) {
+      float mx = -INFINITY;
+      for (int j = tid; j < n; j += kDecThreads) mx = fmaxf(mx, sc[g][j]);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) red_m[warp][g] = mx;
+    }
     __syncthreads();
-    mx = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = ex2(m_run - m_new);  // 0 on the first chunk
-    l_part *= alpha;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] *= alpha;
-    // values of this chunk
+    for (int g = 0; g < G; ++g) {
+      const float mx = fmaxf(fmaxf(red_m[0][g], red_m[1][g]), fmaxf(red_m[2][g], red_m[3][g]));
+      m_new[g] = fmaxf(m_run[g], mx);
+      const float alpha = ex2(m_run[g] - m_new[g]);  // 0 on the first chunk
+      l_part[g] *= alpha;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] *= alpha;
+    }
+    // values of this chunk, each V row slice loaded once for the G heads
     for (int j0 = warp * KPW; j0 < n; j0 += UNR * KPB) {
       float vf[UNR][8];
 #pragma unroll
@@ -143,34 +183,45 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecPara
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        const float pj = (j < n) ? ex2(sc[j] - m_new) : 0.f;
-        if (c == 0) l_part += pj;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(pj, vf[u][e], acc[e]);
+        for (int g = 0; g < G; ++g) {
+          const float pj = (j < n) ? ex2(sc[g][j] - m_new[g]) : 0.f;
+          if (c == 0) l_part[g] += pj;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pj, vf[u][e], acc[g][e]);
+        }
       }
     }
-    m_run = m_new;
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_run[g] = m_new[g];
     __syncthreads();  // sc and red_m are reused by the next chunk
   }
 
   // reduce over the key slots of a warp (lanes with the same dim slice), then over warps
 #pragma unroll
-  for (int o = LPK; o < 32; o <<= 1) {
+  for (int g = 0; g < G; ++g) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, o);
-  }
-  if (kk == 0) {
+    for (int o = LPK; o < 32; o <<= 1) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red_acc[warp][c * 8 + e] = acc[e];
+      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+      l_part[g] += __shfl_xor_sync(0xffffffffu, l_part[g], o);
+    }
+    if (kk == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red_acc[warp][g][c * 8 + e] = acc[g][e];
+    }
+    if (lane == 0) red_l[warp][g] = l_part[g];
   }
-  if (lane == 0) red_l[warp] = l_part;
   __syncthreads();
-  const float l = red_l[0] + red_l[1] + red_l[2] + red_l[3];
-  const float inv_l = 1.f / l;
-  for (int d = tid; d < D; d += kDecThreads)
-    wo[d] = (red_acc[0][d] + red_acc[1][d] + red_acc[2][d] + red_acc[3][d]) * inv_l;
-  if (tid == 0) *wl = (m_run + lg2(l)) * kLn2;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float l = red_l[0][g] + red_l[1][g] + red_l[2][g] + red_l[3][g];
+    const float inv_l = 1.f / l;
+    float* wo = ws_o(g);
+    for (int d = tid; d < D; d += kDecThreads)
+      wo[d] = (red_acc[0][g][d] + red_acc[1][g][d] + red_acc[2][g][d] + red_acc[3][g][d]) * inv_l;
+    if (tid == 0) *ws_l(g) = (m_run[g] + lg2(l)) * kLn2;
+  }
 }
 
 template <bool kFp16, int D, bool kOutF32>
@@ -186,16 +237,17 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecParams p) 
   for (int s = lane; s < p.S; s += 32) mx = fmaxf(mx, wl[s] * kLog2e);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const bool empty = (mx == -INFINITY);  // no split saw a key (warp-uniform)
   float wsum = 0.f;
   for (int s = lane; s < p.S; s += 32) wsum += ex2(wl[s] * kLog2e - mx);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  const float inv = 1.f / wsum;
+  const float inv = empty ? 0.f : 1.f / wsum;
 
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int s = 0; s < p.S; ++s) {
+  for (int s = 0; s < p.S && !empty; ++s) {
     const float w = ex2(wl[s] * kLog2e - mx) * inv;
     const float* row = wo + static_cast<size_t>(s) * D + lane * PER;
     if constexpr (PER == 4) {
@@ -223,12 +275,21 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecParams p) 
       *out = pack2<kFp16>(acc[0], acc[1]);
     }
   }
-  if (lane == 0) p.lse[bh] = (mx + lg2(wsum)) * kLn2;
+  if (lane == 0) p.lse[bh] = empty ? -INFINITY : (mx + lg2(wsum)) * kLn2;
+}
+
+template <bool kFp16, int D, int G>
+void launch_split(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
+  decode_split_kernel<kFp16, D, G><<<dim3(p.Hkv * (p.group / G), a.S, a.B), kDecThreads, 0, stream>>>(p);
 }
 
 template <bool kFp16, int D>
 int launch_decode_t(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
-  decode_split_kernel<kFp16, D><<<dim3(a.H, a.S, a.B), kDecThreads, 0, stream>>>(p);
+  // query heads per CTA: the largest of 8, 4, 2, 1 that divides the group
+  if (p.group % 8 == 0) launch_split<kFp16, D, 8>(a, p, stream);
+  else if (p.group % 4 == 0) launch_split<kFp16, D, 4>(a, p, stream);
+  else if (p.group % 2 == 0) launch_split<kFp16, D, 2>(a, p, stream);
+  else launch_split<kFp16, D, 1>(a, p, stream);
   const int nbh = a.B * a.H;
   const dim3 cgrid((nbh + 3) / 4);
   if (a.o_fp32)
@@ -244,7 +305,11 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   DecParams p;
   p.q = a.q; p.k = a.k; p.v = a.v; p.o = a.o; p.lse = a.lse;
   p.ws_o = a.ws_o; p.ws_lse = a.ws_lse;
+  p.seqlens_k = a.seqlens_k;
+  p.status = a.status;
   p.B = a.B; p.H = a.H; p.Nk = a.Nk; p.S = a.S;
+  p.Hkv = a.Hkv > 0 ? a.Hkv : a.H;
+  p.group = a.H / p.Hkv;
   p.scale_log2 = a.scale * kLog2e;
   if (a.D == 64) return a.fp16 ? launch_decode_t<true, 64>(a, p, stream) : launch_decode_t<false, 64>(a, p, stream);
   return a.fp16 ? launch_decode_t<true, 128>(a, p, stream) : launch_decode_t<false, 128>(a, p, stream);

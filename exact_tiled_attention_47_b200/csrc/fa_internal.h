@@ -32,10 +32,12 @@ struct DecodeArgs {
   float* ws_o;    // [B, H, S, D]
   float* ws_lse;  // [B, H, S]
   int* status;
-  int B, H, Nk, D, S;
+  int B, H, Nk, D, S;  // H: query heads
   float scale;
   int fp16;
   int o_fp32;
+  int Hkv = 0;                     // KV heads (0: same as H); H is a multiple of it
+  const int* seqlens_k = nullptr;  // device int32[B]: valid cache length per batch item (nullptr: Nk)
 };
 
 // Return a cudaError_t-compatible code (0 = success).

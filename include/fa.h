@@ -50,7 +50,7 @@ typedef enum {
   FA_ERR_HEADDIM = 3,     /* D not in {64, 128}                                               */
   FA_ERR_SHAPE = 4,       /* B, H, Nq, Nk, num_splits out of range, or scale not finite > 0   */
   FA_ERR_ALIGN = 5,       /* a tensor pointer is not 16-byte aligned (lse: 4-byte)            */
-  FA_ERR_CU_SEQLENS = 6,  /* cu_seqlens inconsistent with the packed extent (device-detected) */
+  FA_ERR_CU_SEQLENS = 6,  /* cu_seqlens / seqlens_k out of range (device-detected)              */
   FA_ERR_WORKSPACE = 7,   /* decode workspace missing or smaller than required                */
   FA_ERR_DEVICE = 8,      /* no CUDA device, or the current device is not sm_100             */
   FA_ERR_LAUNCH = 9,      /* a CUDA launch or driver call failed                              */
@@ -120,9 +120,10 @@ size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits);
  * exactly how the per-split partial results are combined.
  *
  * q [B, 1, H, D]; k_cache, v_cache [B, Nk, H, D]; o [B, 1, H, D] of type o_dtype; lse [B, H].
- * The query attends to all Nk cached keys (no mask).  The keys are cut into num_splits ranges of
- * ceil(Nk / num_splits) keys; a first kernel writes each range's normalised partial output and
- * partial LSE to `workspace`, a second kernel merges them.  1 <= num_splits <= 128.
+ * The query attends to all Nk cached keys (no mask).  The keys are cut into ranges of
+ * max(ceil(Nk / num_splits), 512) keys (at most num_splits of them; fewer when the cache is short);
+ * a first kernel writes each range's normalised partial output and partial LSE to `workspace`, a
+ * second kernel merges them.  1 <= num_splits <= 128.
  * workspace: device buffer of at least fa_decode_workspace_bytes(B, H, D, num_splits) bytes, owned
  * by the caller, 16-byte aligned; its contents on entry are irrelevant.
  * Returns FA_OK or an fa_status error code.
@@ -131,6 +132,28 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, v
                       int B, int H, int Nk, int D, float scale, int num_splits,
                       void* workspace, size_t workspace_bytes, fa_stream_t stream,
                       int in_dtype, int o_dtype);
+
+/*
+ * fa_decode_splitkv_gqa -- fa_decode_splitkv with grouped KV heads and per-sequence cache lengths.
+ *
+ * Passage: as fa_decode_splitkv.  "Was FlashAttention bei Transformer-Inference verändert" asks
+ * whether a backend supports the cache layout without fixing one; this entry point takes the
+ * common layout with fewer KV heads than query heads and a valid length per sequence.
+ *
+ * q [B, 1, Hq, D]; k_cache, v_cache [B, Nk, Hkv, D] (Nk = cache capacity); o [B, 1, Hq, D] of type
+ * o_dtype; lse [B, Hq].  Hq must be a multiple of Hkv (else FA_ERR_SHAPE); query head h reads KV
+ * head h / (Hq / Hkv).  seqlens_k: device int32[B] (4-byte aligned) or NULL; the query of batch
+ * item b attends to cached keys [0, seqlens_k[b]) (all Nk when NULL).  A length of 0 gives O = 0 and
+ * LSE = -inf; a length outside [0, Nk] is detected on the device, treated as 0, and sets the device
+ * status to FA_ERR_CU_SEQLENS.  Each KV row is read once for all query heads of its group (up to 8
+ * per CTA).  workspace: at least fa_decode_workspace_bytes(B, Hq, D, num_splits) bytes.  Other
+ * arguments, ownership and errors as fa_decode_splitkv; with Hkv = Hq and seqlens_k = NULL the
+ * result equals fa_decode_splitkv's.
+ */
+int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Nk, int D, float scale, int num_splits,
+                          const int* seqlens_k, void* workspace, size_t workspace_bytes,
+                          fa_stream_t stream, int in_dtype, int o_dtype);
 
 /*
  * fa_decode_splitkv_noalloc -- fa_decode_splitkv without a caller-provided workspace.

@@ -39,6 +39,9 @@ CONFIGS = {
                    causal=False, seed=4),
     "decode": dict(B=64, Nk=8192, H=32, D=128, dtype="bf16", scale=1.0 / math.sqrt(128),
                    num_splits=16, seed=5),
+    # grouped KV heads (4 query heads per KV head) and per-sequence cache lengths U{1024..8192}
+    "decode_gqa": dict(B=64, Nk=8192, H=32, Hkv=8, D=128, dtype="bf16", scale=1.0 / math.sqrt(128),
+                       num_splits=16, seed=6, len_lo=1024, len_hi=8192),
 }
 
 
@@ -157,6 +160,14 @@ def varlen_qkv(seed: int, lengths, H: int, D: int, dtype: str, std: float = 1.0)
 def decode_inputs(seed: int, B: int, Nk: int, H: int, D: int, dtype: str, std: float = 1.0):
     """Single-query Q [B,1,H,D] and a K/V cache [B,Nk,H,D], uint16 bits."""
     return dense_qkv(seed, B, 1, Nk, H, D, dtype, std)
+
+
+def decode_gqa_inputs(seed: int, B: int, Nk: int, Hq: int, Hkv: int, D: int, dtype: str, std: float = 1.0):
+    """Single-query Q [B,1,Hq,D] and a K/V cache [B,Nk,Hkv,D], uint16 bits."""
+    q = batched(seed, Q_ID, B, (1, Hq, D), dtype, std)
+    k = batched(seed, K_ID, B, (Nk, Hkv, D), dtype, std)
+    v = batched(seed, V_ID, B, (Nk, Hkv, D), dtype, std)
+    return q, k, v
 
 
 def config_inputs(name: str, **overrides):

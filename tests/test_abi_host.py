@@ -138,6 +138,21 @@ def test_decode_validation_codes(lib):
     assert _dec(lib, ws=A + 8, wsb=need) == fa.FA_ERR_ALIGN
 
 
+def test_decode_gqa_validation_codes(lib):
+    def gqa(Hq=8, Hkv=2, sl=None, wsb=1 << 20, ws=A, **kw):
+        a = dict(q=A, k=A, v=A, o=A, lse=A, B=2, Nk=64, D=128, scale=0.1, S=4)
+        a.update(kw)
+        return lib.fa_decode_splitkv_gqa(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], Hq, Hkv, a["Nk"], a["D"],
+                                         a["scale"], a["S"], sl, ws, wsb, None, 0, 0)
+    assert gqa(Hkv=0) == fa.FA_ERR_SHAPE
+    assert gqa(Hkv=3) == fa.FA_ERR_SHAPE          # 8 query heads are not a multiple of 3
+    assert gqa(Hq=2, Hkv=4) == fa.FA_ERR_SHAPE     # more KV heads than query heads
+    assert gqa(sl=A + 2) == fa.FA_ERR_ALIGN
+    assert gqa(q=None) == fa.FA_ERR_NULL
+    need = fa.fa_decode_workspace_bytes(2, 8, 128, 4)  # sized by the query heads
+    assert gqa(wsb=need - 1) == fa.FA_ERR_WORKSPACE
+
+
 def test_device_status_null(lib):
     assert lib.fa_device_status(None, 0) == fa.FA_ERR_NULL
 
@@ -148,6 +163,7 @@ def test_no_device_is_reported(lib):
     assert _fwd(lib) == fa.FA_ERR_DEVICE
     assert lib.fa_fwd_prefix(A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 10, None, None, 0, 0) == fa.FA_ERR_DEVICE
     assert _dec(lib) == fa.FA_ERR_DEVICE
+    assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     out = ctypes.c_int(0)
     assert lib.fa_device_status(ctypes.byref(out), 0) == fa.FA_ERR_DEVICE
 
