@@ -66,7 +66,7 @@ def measured_traffic(key, scale=1.0):
                 h.update(fh.read())
         if h.hexdigest()[:16] != ent["source_sha"]:
             return None
-        b = ent.get("dram_bytes", ent.get("dram_bytes_per_batch_item"))
+        b = ent.get("dram_bytes", ent.get("dram_bytes_per_batch_item", ent.get("dram_bytes_per_valid_kv_byte")))
         return float(b) * scale
     except (OSError, KeyError, ValueError):
         return None
@@ -522,6 +522,7 @@ def main():
                                  "valid_kv_bytes": kv_g},
                       "roofline": {"bound": "hbm", "achieved": gbs_g, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                    "frac": gbs_g / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy",
+                                   "traffic": measured_traffic("decode_gqa", kv_g),
                                    "algorithmic_bytes_per_step": alg_g},
                       "gpu_launches": 2 * dsteps}
         del qg, kg, vg, og, lg_, wsg, sl
