@@ -13,16 +13,19 @@ Modules:
                 inside, running max m and running sum l), and the pairwise merge of softmax
                 statistics of key groups, including the split-KV partial/combine form.
   brute      -- scalar pure-Python (math.fsum) evaluation for tiny inputs.
+  backward   -- dQ, dK, dV: the derivative of the forward definition for an upstream gradient dO.
 """
 from .attention import (attention_head, attention_dense, attention_varlen, attention_rows,
                         attention_decode, attention_decode_gqa, padded_key_mask_attention)
 from .online import (tiled_online_attention, group_stats, merge_groups, softmax_by_groups,
                      split_kv_partials, combine_partials)
 from .brute import brute_attention_head
+from .backward import attention_head_backward, attention_dense_backward, backward_row_terms
 
 __all__ = [
     "attention_head", "attention_dense", "attention_varlen", "attention_rows", "attention_decode",
     "attention_decode_gqa",
     "padded_key_mask_attention", "tiled_online_attention", "group_stats", "merge_groups",
     "softmax_by_groups", "split_kv_partials", "combine_partials", "brute_attention_head",
+    "attention_head_backward", "attention_dense_backward", "backward_row_terms",
 ]

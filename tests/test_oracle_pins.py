@@ -23,7 +23,9 @@ wrong LSE base, a bad group merge) fails at least one of them:
     is bidirectional), brute force, the row sampler and the packed varlen form;
   * decode with grouped KV heads and per-sequence cache lengths: equal to the dense decode over KV
     heads repeated G times, equal to decode over the truncated cache, the Q = 0 closed form, and
-    the split-KV combine with empty splits.
+    the split-KV combine with empty splits;
+  * the backward (dQ, dK, dV): central finite differences of the forward oracle, the Q = 0 closed
+    forms, invariance of dQ and dV under a common key shift, and zero total dK.
 """
 import json
 import math
@@ -447,3 +449,62 @@ def test_combine_of_empty_splits():
     o_ref, lse_ref = oracle.attention_head(q[None, :], k, v, 0.4)
     np.testing.assert_allclose(o, o_ref[0], rtol=1e-12, atol=1e-14)
     assert abs(lse - lse_ref[0]) < 1e-12
+
+
+# ---------------------------------------------------------------------------------------------
+# backward: the derivative of the forward definition
+
+
+def _loss(q, k, v, do, scale, causal):
+    o, _ = oracle.attention_head(q, k, v, scale, causal)
+    return float((o * do).sum())
+
+
+@pytest.mark.parametrize("nq,nk,causal", [(6, 6, False), (7, 7, True), (5, 9, True), (9, 5, True), (4, 11, False)])
+def test_backward_matches_finite_differences(nq, nk, causal):
+    # central differences of the (pinned) forward oracle: error O(h^2) ~ 1e-10 for h = 1e-5
+    d, dv_, scale, h = 5, 4, 0.4, 1e-5
+    rng = np.random.default_rng(nq * 31 + nk)
+    q, k, v = rng.standard_normal((nq, d)), rng.standard_normal((nk, d)), rng.standard_normal((nk, dv_))
+    do = rng.standard_normal((nq, dv_))
+    dq, dk, dv = oracle.attention_head_backward(q, k, v, do, scale, causal)
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = _loss(q, k, v, do, scale, causal)
+            x[idx] = keep - h
+            lm = _loss(q, k, v, do, scale, causal)
+            x[idx] = keep
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+def test_backward_closed_forms():
+    # Q = 0, no mask: P is uniform 1/Nk, so dV_j = (1/Nk) sum_i dO_i for every key j and
+    # dS_ij = (dO_i . V_j - dO_i . mean(V)) / Nk
+    nq, nk, d = 6, 10, 4
+    rng = np.random.default_rng(5)
+    q = np.zeros((nq, d))
+    k, v, do = rng.standard_normal((nk, d)), rng.standard_normal((nk, d)), rng.standard_normal((nq, d))
+    dq, dk, dv = oracle.attention_head_backward(q, k, v, do, 0.5)
+    np.testing.assert_allclose(dv, np.repeat(do.sum(axis=0, keepdims=True) / nk, nk, axis=0), rtol=1e-13)
+    ds = (do @ v.T - (do @ v.mean(axis=0))[:, None]) / nk
+    np.testing.assert_allclose(dq, 0.5 * ds @ k, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(dk, np.zeros_like(k))  # dK = scale * dS^T Q = 0
+
+
+def test_backward_row_sums_and_shift_invariance():
+    # adding a vector c to every key shifts each score row by a constant, so P, dS and dV are
+    # unchanged and dQ = scale dS (K + c) changes by scale (sum_j dS_ij) c = 0: dS rows sum to zero
+    nq, nk, d = 8, 12, 5
+    rng = np.random.default_rng(6)
+    q, k, v, do = (rng.standard_normal(s) for s in ((nq, d), (nk, d), (nk, d), (nq, d)))
+    dq, dk, dv = oracle.attention_head_backward(q, k, v, do, 0.3)
+    c = rng.standard_normal(d)
+    dq2, dk2, dv2 = oracle.attention_head_backward(q, k + c, v, do, 0.3)
+    np.testing.assert_allclose(dq2, dq, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(dv2, dv, rtol=1e-11, atol=1e-13)
+    # total gradient wrt a key shift: sum_j dK_j = scale * sum_ij dS_ij q_i = 0
+    np.testing.assert_allclose(dk.sum(axis=0), np.zeros(d), atol=1e-12)
