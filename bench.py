@@ -339,6 +339,38 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
                   "roofline": {"bound": "tensor", "achieved": ptf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                                "frac": ptf / pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst"},
                   "gpu_launches": psteps}
+    # the backward pass on the same inputs (upstream gradient: seeded, tensor id 3)
+    bwd = None
+    if not args.no_backward:
+        dout = to_dev(si.batched(seed, 3, B, (N, H, D), dt), dt, dev)
+        gq, gk, gv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+        wsb = fa.fa_bwd_workspace_bytes(B, H, N)
+        wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        step()  # od, lse of these inputs
+
+        def bstep():
+            st = fa.fa_bwd(qd, kd, vd, od, dout, lse, gq, gk, gv, B, H, N, N, D, scale, causal, wsd, wsb, stream)
+            if st:
+                raise fa.FAError(st, "fa_bwd")
+
+        for _ in range(args.warmup):
+            bstep()
+        bsteps = max(10, min(args.steps, 50))
+        ms_b = timed(bstep, bsteps, stream, dist)
+        if fa.fa_device_status(clear=True) != 0:
+            raise RuntimeError("device status set during the timed backward run")
+        bf = 2.5 * prefill_flops(B, H, N, N, D, causal)  # dV, dP, dQ, dK and the recomputed S
+        btf = bf / (ms_b / bsteps * 1e-3) / 1e12
+        bwd = {"metric": "attention bwd TFLOPS", "value": whole_job_rate(bf, ms_b / bsteps, world) / 1e12,
+               "unit": "TFLOP/s", "ms_per_step": ms_b / bsteps, "steps": bsteps,
+               "algorithmic_flops_per_step": bf,
+               "note": "FLOPs counted as 2.5x the forward (five GEMMs); the kernels run seven (S and dP "
+                       "are recomputed in both the dQ and the dK/dV kernel)",
+               "roofline": {"bound": "tensor", "achieved": btf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                            "frac": btf / pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst"},
+               "gpu_launches": 3 * bsteps}
+        del dout, gq, gk, gv, wsd
+
     flops_step = prefill_flops(B, H, N, N, D, causal)
     ms_step = ms / args.steps
     tflops_rank = flops_step / (ms_step * 1e-3) / 1e12
@@ -380,7 +412,7 @@ def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
     del qd, kd, vd, od, lse
     torch.cuda.empty_cache()
 
-    return value, ms_step, roof, e2e, clk, prefix
+    return value, ms_step, roof, e2e, clk, prefix, bwd
 
 
 def main():
@@ -392,6 +424,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefix", action="store_true", help="skip the prefix-mask timing of the prefill inputs")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing of the prefill inputs")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
@@ -431,11 +464,11 @@ def main():
     scale = cfg["scale"]
     stream = torch.cuda.current_stream(dev)
     value = ms_step = None
-    roof = e2e = prefix = None
+    roof = e2e = prefix = bwd = None
     clk = ClockSampler(local)
     if run_prefill:
-        value, ms_step, roof, e2e, clk, prefix = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa,
-                                                             torch)
+        value, ms_step, roof, e2e, clk, prefix, bwd = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind,
+                                                                  fa, torch)
 
     # ---------------- decode (secondary metric) ----------------
     dec = None
@@ -551,7 +584,7 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof, "clocks": clk.summary(), "e2e": e2e,
         "gpu_launches": args.steps if run_prefill else 0,
-        "decode": dec, "prefix": prefix, "cpu_baseline": cpu,
+        "decode": dec, "prefix": prefix, "backward": bwd, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     return 0

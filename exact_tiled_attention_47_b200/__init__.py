@@ -18,7 +18,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
  FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT) = range(11)
 
 __all__ = [
-    "fa_fwd", "fa_fwd_prefix", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
+    "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
@@ -76,6 +76,25 @@ def fa_fwd_prefix(q, k, v, o, lse, B, H, Nq, Nk, D, scale, prefix_len, cu_seqlen
     return lib.fa_fwd_prefix(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(H), int(Nq), int(Nk),
                              int(D), float(scale), int(prefix_len), _ptr(cu_seqlens), _stream(stream),
                              int(in_dtype), int(o_dtype))
+
+
+def fa_bwd_workspace_bytes(B, H, Nq) -> int:
+    return int(load().fa_bwd_workspace_bytes(int(B), int(H), int(Nq)))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, workspace, workspace_bytes=None,
+           stream=None, in_dtype=None, grad_dtype=None) -> int:
+    """Marshal to the C ``fa_bwd``; returns its status.  Dtypes default to those of q and dq."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if grad_dtype is None:
+        grad_dtype = _dtype_code(dq)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                      int(B), int(H), int(Nq), int(Nk), int(D), float(scale), int(bool(causal)), _ptr(workspace),
+                      int(workspace_bytes), _stream(stream), int(in_dtype), int(grad_dtype))
 
 
 def fa_decode_workspace_bytes(B, H, D, num_splits) -> int:
@@ -187,6 +206,24 @@ def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None
     if st != FA_OK:
         raise FAError(st, "fa_fwd_prefix" if prefix_len is not None else "fa_fwd")
     return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal=False, scale=None, grad_dtype=None, stream=None):
+    """dQ, dK, dV for dense q [B,Nq,H,D], k/v [B,Nk,H,D], the forward o / lse and the upstream dout."""
+    import torch
+    B, Nq, H, D = q.shape
+    Nk = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    grad_dtype = q.dtype if grad_dtype is None else grad_dtype
+    dq = torch.empty(q.shape, device=q.device, dtype=grad_dtype)
+    dk = torch.empty(k.shape, device=q.device, dtype=grad_dtype)
+    dv = torch.empty(v.shape, device=q.device, dtype=grad_dtype)
+    ws = torch.empty(fa_bwd_workspace_bytes(B, H, Nq), device=q.device, dtype=torch.uint8)
+    st = fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, ws, stream=stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, workspace=None,

@@ -1,0 +1,567 @@
+// fa_backward_sm100.cu -- gradients of exact attention on B200 tensor cores (tcgen05 + TMEM + TMA).
+//
+// "轻松读懂FlashAttention 上", end of section "Softmax求解重构": the forward pass keeps O and the
+// softmax statistics so that the backward pass can recompute S and P instead of reading them back.
+// With the natural-log LSE of the forward pass, P = 2^(S*scale*log2(e) - LSE*log2(e)) needs no
+// running max.  For an upstream gradient dO of L = sum(dO * O) (the derivative of the forward
+// definition):  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Drow) with Drow_i = sum_d dO_id O_id,
+// dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three kernels, no atomics:
+//   bwd_rowterm_kernel  Drow[b,h,i] (fp32), one thread per (b, i, h) row.
+//   bwd_dq_kernel       CTA = one 128-row query tile.  Per key block j: S = Q K_j^T and
+//                       dP = dO V_j^T into TMEM, the four compute warps (thread = query row) form dS
+//                       32 columns at a time and write it (bf16/fp16) over the first 64 columns of
+//                       dP, then dQ += dS K_j accumulates in TMEM.  dQ * scale is written at the end.
+//   bwd_dkdv_kernel     CTA = one 128-row key tile.  Per query block i: S^T = K Q_i^T and
+//                       dP^T = V dO_i^T into TMEM, the compute warps (thread = key row) form P^T and
+//                       dS^T 32 query columns at a time (the block's LSE and Drow come through shared
+//                       memory) and write them over S^T and dP^T, then dV += P^T dO_i and
+//                       dK += dS^T Q_i accumulate in TMEM.  dV and dK * scale are written at the end.
+// Both recompute S and dP (two more GEMMs than the minimum) so that each gradient is owned by one
+// CTA and accumulates in TMEM.  Warps 0-3 compute, warp 4 is the TMA producer, warp 5 owns TMEM and
+// issues every tcgen05.mma from one thread; the next block's S/dP are issued after the products that
+// read the previous block's P/dS columns (the tensor core runs one thread's MMAs in order).  The MMA
+// forms are those of the forward kernel: SS with both operands K-major (S, dP) and TS with the A
+// operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal runs skip fully masked
+// blocks; masking is applied on the blocks that cross the diagonal and at the sequence ends.
+#include <cudaTypedefs.h>
+
+#include "fa_prefill_common.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBT = 128;  // rows per tile (queries or keys)
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
+constexpr int kStages = 2;
+constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256;  // S (P over it), dP (dS over it), accumulators
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kTileBytes = kBT * D * 2;
+  static constexpr int kUsed = (2 + 2 * kStages) * kTileBytes + 2 * kStages * kBT * 4 + 256 + 1024;
+  // at least 120 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
+  static constexpr int kSmemBytes = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+};
+static_assert(BwdCfg<128>::kSmemBytes <= 232448, "shared memory budget");
+
+struct BwdParams {
+  const float* lse;   // [B, H, Nq]
+  const float* drow;  // [B, H, Nq]
+  void* g0;           // dq (dq kernel) or dk (dkdv kernel)
+  void* g1;           // dv (dkdv kernel)
+  int* status;
+  int B, H, Nq, Nk;
+  int num_tiles;  // query tiles (dq) or key tiles (dkdv) per (b, h)
+  float scale, scale_log2;
+  int causal;
+};
+
+struct BwdBars {
+  uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
+  uint64_t st_full[kStages], st_empty[kStages];  // streamed tiles (K + V, or Q + dO + row stats)
+  uint64_t s_full, p_full, o_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(BwdBars) <= 256, "barrier block too large");
+
+// ------------------------------------------------------------------------------------------------
+// Drow = sum_d dO * O per row
+
+template <bool kFp16, int D>
+__global__ void __launch_bounds__(256) bwd_rowterm_kernel(const void* o, const void* dout, float* drow, int B,
+                                                          int H, int N) {
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b, i, h) row
+  if (r >= static_cast<long long>(B) * N * H) return;
+  const uint4* a = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(o) + r * D);
+  const uint4* g = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(dout) + r * D);
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 x = a[c], y = g[c];
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 xf = unpack2<kFp16>(xs[e]), yf = unpack2<kFp16>(ys[e]);
+      acc = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, acc));
+    }
+  }
+  const int h = static_cast<int>(r % H);
+  const long long bi = r / H;
+  const int i = static_cast<int>(bi % N);
+  const int b = static_cast<int>(bi / N);
+  drow[(static_cast<size_t>(b) * H + h) * N + i] = acc;
+}
+
+// ------------------------------------------------------------------------------------------------
+// shared pieces
+
+__device__ __forceinline__ void smem_desc_pair_k(uint32_t a, uint32_t b, int kk, uint64_t& da, uint64_t& db) {
+  // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row; every 4 steps
+  // move to the next 64-column panel.  SBO = 8 rows * 128 B.
+  const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
+  da = smem_desc_sw128(a + off, 16, 1024);
+  db = smem_desc_sw128(b + off, 16, 1024);
+}
+
+template <int D>
+__device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint32_t a, uint32_t b, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint64_t da, db;
+    smem_desc_pair_k(a, b, kk, da, db);
+    mma_ss(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// d += A (TMEM, 128 x 128 packed 16-bit) * B (shared, N-major, 128 rows of D)
+__device__ __forceinline__ void mma_tn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kBT / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, kPanelBytes, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Every lane of the warp loads (tcgen05.ld is warp-collective); only lanes with store write the row.
+template <int D, bool kFp16, bool kOutF32>
+__device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint32_t taddr, float mul, bool store) {
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t r[32];
+    tmem_ld32_sync(taddr + ch * 32, r);
+    if (!store) continue;
+    if constexpr (kOutF32) {
+      float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(out) + row_elem + ch * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        o4[i] = make_float4(__uint_as_float(r[4 * i]) * mul, __uint_as_float(r[4 * i + 1]) * mul,
+                            __uint_as_float(r[4 * i + 2]) * mul, __uint_as_float(r[4 * i + 3]) * mul);
+    } else {
+      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_elem + ch * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float* f = reinterpret_cast<const float*>(r + 8 * i);
+        o4[i] = make_uint4(pack2<kFp16>(f[0] * mul, f[1] * mul), pack2<kFp16>(f[2] * mul, f[3] * mul),
+                           pack2<kFp16>(f[4] * mul, f[5] * mul), pack2<kFp16>(f[6] * mul, f[7] * mul));
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->fixed_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->st_full[s], 1);
+      mbar_init(&bars->st_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+__device__ __forceinline__ void bwd_teardown(BwdBars* bars, int warp, uint32_t tbase) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// dQ: one query tile per CTA, walking the key blocks it sees
+
+template <int D, bool kFp16, bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + C::kTileBytes;
+  auto sK = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
+  auto sV = [&](int st) { return smem + (2 + kStages + st) * C::kTileBytes; };
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * kStages) * C::kTileBytes + 2 * kStages * kBT * 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
+  const int m_block = p.num_tiles - 1 - static_cast<int>(blockIdx.x % p.num_tiles);  // longest first
+  const int b = bh / p.H, h = bh % p.H;
+  const int m0 = m_block * kBT;
+  const int Lq = p.Nq, Lk = p.Nk, diag = Lk - Lq;
+  int kv_end = Lk;
+  if (p.causal) kv_end = min(Lk, m0 + kBT + diag);
+  const int n = (kv_end > 0) ? (kv_end + kBT - 1) / kBT : 0;
+  if (n == 0) {  // no row of the tile sees a key: dQ = 0
+    if (warp < 4) {
+      const int qi = m0 + warp * 32 + lane;
+      if (qi < Lq) {
+        const size_t row = ((static_cast<size_t>(b) * Lq + qi) * p.H + h) * D;
+        for (int d = 0; d < D; ++d) {
+          if constexpr (kOutF32) static_cast<float*>(p.g0)[row + d] = 0.f;
+          else static_cast<uint16_t*>(p.g0)[row + d] = 0;
+        }
+      }
+    }
+    return;
+  }
+  bwd_setup(bars, warp);
+  const uint32_t tbase = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();
+      mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_3d(&tm_q, &bars->fixed_full, sQ + pn * kPanelBytes, pn * 64, h, b * Lq + m0);
+        tma_load_3d(&tm_do, &bars->fixed_full, sDO + pn * kPanelBytes, pn * 64, h, b * Lq + m0);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages;
+        if (!(ok = mbar_wait(&bars->st_empty[st], ((j / kStages) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_3d_hint(&tm_k, &bars->st_full[st], sK(st) + pn * kPanelBytes, pn * 64, h, b * Lk + j * kBT, keep);
+          tma_load_3d_hint(&tm_v, &bars->st_full[st], sV(st) + pn * kPanelBytes, pn * 64, h, b * Lk + j * kBT, keep);
+        }
+        issued = j + 1;
+      }
+      if (!ok) {
+        drain_wait(&bars->fixed_full, 0);
+        for (int j = max(0, issued - kStages); j < issued; ++j) drain_wait(&bars->st_full[j % kStages], (j / kStages) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr int fmt = kFp16 ? 0 : 1;
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+      constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kStages;
+        if (!(ok = mbar_wait(&bars->st_full[st], (j / kStages) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_kk<D>(tbase + kColS, smem_addr(sQ), smem_addr(sK(st)), idesc_s);    // S = Q K_j^T
+        mma_kk<D>(tbase + kColDP, smem_addr(sDO), smem_addr(sV(st)), idesc_s);  // dP = dO V_j^T
+        mma_commit(&bars->s_full);
+        if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_tn(tbase + kColA, tbase + kColDP, smem_addr(sK(st)), idesc_g, j > 0);  // dQ += dS K_j
+        mma_commit(&bars->st_empty[st]);
+        mma_commit(&bars->o_done);
+      }
+      mma_commit(&bars->drain);
+      drain_wait(&bars->drain, 0);
+    }
+  } else {
+    const int r = warp * 32 + lane;
+    const int qi = m0 + r;
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;
+    const int tile_lim = p.causal ? min(Lk, m0 + 1 + diag) : Lk;
+    const size_t stat = (static_cast<size_t>(b) * p.H + h) * Lq + min(qi, Lq - 1);
+    const float lse = p.lse[stat];
+    // rows without keys (LSE = -inf) and rows past the end get P = 0
+    const float lse2 = (qi < Lq && lse != -INFINITY) ? lse * kLog2e : INFINITY;
+    const float dr = (qi < Lq) ? p.drow[stat] : 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!(ok = warp_wait(&bars->s_full, j & 1, abort_flag, p.status))) break;
+      tc_fence_after();
+      const bool masked = (j + 1) * kBT > tile_lim;
+      const int lim = row_lim - j * kBT;
+#pragma unroll
+      for (int ch = 0; ch < kBT / 32; ++ch) {
+        uint32_t s[32], dp[32], pk[16];
+        tmem_ld32_sync(lane_base + kColS + ch * 32, s);
+        tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = ch * 32 + 2 * i;
+          float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, -lse2));
+          float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, -lse2));
+          if (masked) {
+            if (c0 >= lim) p0 = 0.f;
+            if (c0 + 1 >= lim) p1 = 0.f;
+          }
+          pk[i] = pack2<kFp16>(p0 * (__uint_as_float(dp[2 * i]) - dr), p1 * (__uint_as_float(dp[2 * i + 1]) - dr));
+        }
+        tmem_st16(lane_base + kColDP + ch * 16, pk);  // dS over dP, below the unread columns
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = warp_wait(&bars->o_done, (n - 1) & 1, abort_flag, p.status);
+    if (ok) {
+      tc_fence_after();
+      const size_t row = (static_cast<size_t>(b) * Lq + min(qi, Lq - 1)) * p.H + h;
+      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq);
+    }
+  }
+  bwd_teardown(bars, warp, tbase);
+}
+
+// ------------------------------------------------------------------------------------------------
+// dK, dV: one key tile per CTA, walking the query blocks that see it
+
+template <int D, bool kFp16, bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + C::kTileBytes;
+  auto sQ = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
+  auto sDO = [&](int st) { return smem + (2 + kStages + st) * C::kTileBytes; };
+  float* sStat = reinterpret_cast<float*>(smem + (2 + 2 * kStages) * C::kTileBytes);  // [stage][lse2 | drow][128]
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * kStages) * C::kTileBytes + 2 * kStages * kBT * 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
+  const int n_block = static_cast<int>(blockIdx.x % p.num_tiles);  // causal: the first key tile sees most
+  const int b = bh / p.H, h = bh % p.H;
+  const int n0 = n_block * kBT;
+  const int Lq = p.Nq, Lk = p.Nk, diag = Lk - Lq;
+  // query blocks that see any key of this tile: q >= k - diag for the tile's first key k = n0
+  const int i_first = p.causal ? max(0, n0 - diag) / kBT : 0;
+  const int nq_blocks = (Lq + kBT - 1) / kBT;
+  const int n = (p.causal && n0 - diag > Lq - 1) ? 0 : nq_blocks - i_first;
+  if (n <= 0) {  // no query sees this tile: dK = dV = 0
+    if (warp < 4) {
+      const int kj = n0 + warp * 32 + lane;
+      if (kj < Lk) {
+        const size_t row = ((static_cast<size_t>(b) * Lk + kj) * p.H + h) * D;
+        for (int d = 0; d < D; ++d) {
+          if constexpr (kOutF32) {
+            static_cast<float*>(p.g0)[row + d] = 0.f;
+            static_cast<float*>(p.g1)[row + d] = 0.f;
+          } else {
+            static_cast<uint16_t*>(p.g0)[row + d] = 0;
+            static_cast<uint16_t*>(p.g1)[row + d] = 0;
+          }
+        }
+      }
+    }
+    return;
+  }
+  bwd_setup(bars, warp);
+  const uint32_t tbase = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (warp == kProducerWarp) {
+    const uint64_t keep = l2_policy_evict_last();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_3d(&tm_k, &bars->fixed_full, sK + pn * kPanelBytes, pn * 64, h, b * Lk + n0);
+        tma_load_3d(&tm_v, &bars->fixed_full, sV + pn * kPanelBytes, pn * 64, h, b * Lk + n0);
+      }
+    }
+    int issued = 0;
+    bool ok = true;
+    for (int jj = 0; jj < n; ++jj) {
+      const int i = i_first + jj, st = jj % kStages;
+      if (!(ok = warp_wait(&bars->st_empty[st], ((jj / kStages) & 1) ^ 1, abort_flag, p.status))) break;
+      // the block's LSE (log2 units; +inf for rows without keys or past the end, so P = 0) and Drow
+      float* stat = sStat + st * 2 * kBT;
+      const size_t base = (static_cast<size_t>(b) * p.H + h) * Lq;
+      for (int c = lane; c < kBT; c += 32) {
+        const int qi = i * kBT + c;
+        float l2 = INFINITY, dr = 0.f;
+        if (qi < Lq) {
+          const float lse = p.lse[base + qi];
+          if (lse != -INFINITY) l2 = lse * kLog2e;
+          dr = p.drow[base + qi];
+        }
+        stat[c] = l2;
+        stat[kBT + c] = dr;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);  // release orders the stores above
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_3d_hint(&tm_q, &bars->st_full[st], sQ(st) + pn * kPanelBytes, pn * 64, h, b * Lq + i * kBT, keep);
+          tma_load_3d_hint(&tm_do, &bars->st_full[st], sDO(st) + pn * kPanelBytes, pn * 64, h, b * Lq + i * kBT, keep);
+        }
+      }
+      issued = jj + 1;
+    }
+    if (!ok && lane == 0) {
+      drain_wait(&bars->fixed_full, 0);
+      for (int jj = max(0, issued - kStages); jj < issued; ++jj) drain_wait(&bars->st_full[jj % kStages], (jj / kStages) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr int fmt = kFp16 ? 0 : 1;
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+      constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status);
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const int st = jj % kStages;
+        if (!(ok = mbar_wait(&bars->st_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_kk<D>(tbase + kColS, smem_addr(sK), smem_addr(sQ(st)), idesc_s);    // S^T = K Q_i^T
+        mma_kk<D>(tbase + kColDP, smem_addr(sV), smem_addr(sDO(st)), idesc_s);  // dP^T = V dO_i^T
+        mma_commit(&bars->s_full);
+        if (!(ok = mbar_wait(&bars->p_full, jj & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_tn(tbase + kColA, tbase + kColS, smem_addr(sDO(st)), idesc_g, jj > 0);      // dV += P^T dO_i
+        mma_tn(tbase + kColA + D, tbase + kColDP, smem_addr(sQ(st)), idesc_g, jj > 0);  // dK += dS^T Q_i
+        mma_commit(&bars->st_empty[st]);
+        mma_commit(&bars->o_done);
+      }
+      mma_commit(&bars->drain);
+      drain_wait(&bars->drain, 0);
+    }
+  } else {
+    const int r = warp * 32 + lane;
+    const int kj = n0 + r;  // this thread's key
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int jj = 0; jj < n; ++jj) {
+      const int i = i_first + jj, st = jj % kStages;
+      if (!(ok = warp_wait(&bars->s_full, jj & 1, abort_flag, p.status))) break;
+      // the stage's LSE/Drow: the producer stored them before its arrival on st_full (already
+      // complete here; this stage cannot be refilled before this block's P V products)
+      if (!(ok = warp_wait(&bars->st_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
+      tc_fence_after();
+      const float* stat = sStat + st * 2 * kBT;
+      // key kj is visible to query q iff q >= kj - diag (causal); whole block visible iff its first
+      // query already sees the tile's last key
+      const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
+      const int q_lo = kj - diag - i * kBT;  // columns c < q_lo are masked
+#pragma unroll
+      for (int ch = 0; ch < kBT / 32; ++ch) {
+        uint32_t s[32], dp[32], pk[16], dk[16];
+        tmem_ld32_sync(lane_base + kColS + ch * 32, s);
+        tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 l2 = *reinterpret_cast<const float4*>(stat + ch * 32 + 4 * q4);
+          const float4 dr = *reinterpret_cast<const float4*>(stat + kBT + ch * 32 + 4 * q4);
+          const float lv[4] = {l2.x, l2.y, l2.z, l2.w}, dv[4] = {dr.x, dr.y, dr.z, dr.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = ch * 32 + 4 * q4 + e;
+            float pe = ex2(fmaf(__uint_as_float(s[4 * q4 + e]), sl2, -lv[e]));
+            if (masked && c < q_lo) pe = 0.f;
+            pv[e] = pe;
+            dsv[e] = pe * (__uint_as_float(dp[4 * q4 + e]) - dv[e]);
+          }
+          pk[2 * q4] = pack2<kFp16>(pv[0], pv[1]);
+          pk[2 * q4 + 1] = pack2<kFp16>(pv[2], pv[3]);
+          dk[2 * q4] = pack2<kFp16>(dsv[0], dsv[1]);
+          dk[2 * q4 + 1] = pack2<kFp16>(dsv[2], dsv[3]);
+        }
+        tmem_st16(lane_base + kColS + ch * 16, pk);   // P^T over S^T, below the unread columns
+        tmem_st16(lane_base + kColDP + ch * 16, dk);  // dS^T over dP^T
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = warp_wait(&bars->o_done, (n - 1) & 1, abort_flag, p.status);
+    if (ok) {
+      tc_fence_after();
+      const size_t row = ((static_cast<size_t>(b) * Lk + min(kj, Lk - 1)) * p.H + h) * D;
+      store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk);         // dV
+      store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk);  // dK
+    }
+  }
+  bwd_teardown(bars, warp, tbase);
+}
+
+template <int D, bool kFp16, bool kOutF32>
+int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, cudaStream_t stream) {
+  const int smem = BwdCfg<D>::kSmemBytes;
+  const size_t rows = static_cast<size_t>(a.B) * a.Nq * a.H;
+  bwd_rowterm_kernel<kFp16, D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(a.o, a.dout, a.drow,
+                                                                                             a.B, a.H, a.Nq);
+  auto kq = bwd_dq_kernel<D, kFp16, kOutF32>;
+  cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  auto kkv = bwd_dkdv_kernel<D, kFp16, kOutF32>;
+  e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  BwdParams pq = p;
+  pq.g0 = a.dq;
+  pq.num_tiles = (a.Nq + kBT - 1) / kBT;
+  kq<<<static_cast<unsigned>(pq.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pq);
+  BwdParams pk = p;
+  pk.g0 = a.dk;
+  pk.g1 = a.dv;
+  pk.num_tiles = (a.Nk + kBT - 1) / kBT;
+  kkv<<<static_cast<unsigned>(pk.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pk);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_backward(const BackwardArgs& a, cudaStream_t stream) {
+  CUtensorMap m[4];
+  if (!make_tma_map(&m[0], a.q, a.B * a.Nq, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[1], a.dout, a.B * a.Nq, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[2], a.k, a.B * a.Nk, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[3], a.v, a.B * a.Nk, a.H, a.D, a.fp16, kBT))
+    return static_cast<int>(cudaErrorInvalidValue);
+  BwdParams p;
+  p.lse = a.lse;
+  p.drow = a.drow;
+  p.g0 = p.g1 = nullptr;
+  p.status = a.status;
+  p.B = a.B;
+  p.H = a.H;
+  p.Nq = a.Nq;
+  p.Nk = a.Nk;
+  p.num_tiles = 0;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+  p.causal = a.causal ? 1 : 0;
+  if (a.D == 64) {
+    if (a.fp16) return a.g_fp32 ? launch_bwd_t<64, true, true>(a, m, p, stream) : launch_bwd_t<64, true, false>(a, m, p, stream);
+    return a.g_fp32 ? launch_bwd_t<64, false, true>(a, m, p, stream) : launch_bwd_t<64, false, false>(a, m, p, stream);
+  }
+  if (a.fp16) return a.g_fp32 ? launch_bwd_t<128, true, true>(a, m, p, stream) : launch_bwd_t<128, true, false>(a, m, p, stream);
+  return a.g_fp32 ? launch_bwd_t<128, false, true>(a, m, p, stream) : launch_bwd_t<128, false, false>(a, m, p, stream);
+}
+
+}  // namespace fa

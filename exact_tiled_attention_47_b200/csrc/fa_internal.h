@@ -40,9 +40,29 @@ struct DecodeArgs {
   const int* seqlens_k = nullptr;  // device int32[B]: valid cache length per batch item (nullptr: Nk)
 };
 
+struct BackwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;     // forward output, input type
+  const void* dout;  // upstream gradient, input type
+  const float* lse;  // forward LSE [B, H, Nq]
+  void* dq;
+  void* dk;
+  void* dv;
+  float* drow;  // workspace: [B, H, Nq] fp32
+  int* status;
+  int B, H, Nq, Nk, D;
+  float scale;
+  int causal;
+  int fp16;    // input type: 1 = fp16, 0 = bf16
+  int g_fp32;  // gradient type: 1 = fp32, 0 = input type
+};
+
 // Return a cudaError_t-compatible code (0 = success).
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int launch_backward(const BackwardArgs& a, cudaStream_t stream);
 
 int* device_status_ptr();  // address of this device's status word (nullptr on failure)
 int check_device(int* dev_out);  // FA_OK if the current device is sm_100, else FA_ERR_DEVICE

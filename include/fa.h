@@ -105,6 +105,34 @@ int fa_fwd_prefix(const void* q, const void* k, const void* v, void* o, float* l
                   const int* cu_seqlens, fa_stream_t stream, int in_dtype, int o_dtype);
 
 /*
+ * fa_bwd_workspace_bytes -- size of the scratch buffer fa_bwd needs: B * H * Nq * 4 bytes (one fp32
+ * row term per query), rounded up to 256 bytes.  Returns 0 for invalid arguments.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq);
+
+/*
+ * fa_bwd -- gradients dQ, dK, dV of the attention forward pass (dense layout).
+ *
+ * Passage: "轻松读懂FlashAttention 上", end of section "Softmax求解重构": keeping O and the softmax
+ * statistics lets the backward pass recompute S and P instead of storing them; the Hugging Face
+ * page's parameter table (row training) ties training mode to gradient computation.  The gradients
+ * are the derivative of fa_fwd's definition for an upstream gradient dO of L = sum(dO * O):
+ * dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q, with P
+ * recomputed from Q, K and the forward LSE.
+ *
+ * q, o, dout [B, Nq, H, D] and k, v [B, Nk, H, D] of in_dtype (FA_BF16 / FA_FP16); lse [B, H, Nq]
+ * fp32 as written by fa_fwd with the same q, k, v, scale and causal; dq [B, Nq, H, D] and dk, dv
+ * [B, Nk, H, D] of grad_dtype (in_dtype or FA_FP32), fully overwritten.  causal as fa_fwd
+ * (bottom-right aligned).  workspace: device buffer of at least fa_bwd_workspace_bytes(B, H, Nq)
+ * bytes, owned by the caller, 16-byte aligned.  No varlen or prefix form.  Limits and errors as
+ * fa_fwd (FA_ERR_WORKSPACE for a missing or short workspace).  A query row with LSE = -inf (no
+ * visible key) contributes nothing.  Three kernels run in order on `stream`; nothing is allocated.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal,
+           void* workspace, size_t workspace_bytes, fa_stream_t stream, int in_dtype, int grad_dtype);
+
+/*
  * fa_decode_workspace_bytes -- size of the scratch buffer fa_decode_splitkv needs:
  * num_splits * B * H * (D + 1) * 4 bytes (one fp32 partial output row and one fp32 partial LSE per
  * split), rounded up to 256 bytes.  Returns 0 for invalid arguments.

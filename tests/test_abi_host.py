@@ -153,6 +153,27 @@ def test_decode_gqa_validation_codes(lib):
     assert gqa(wsb=need - 1) == fa.FA_ERR_WORKSPACE
 
 
+def test_bwd_validation_codes(lib):
+    def bwd(**kw):
+        a = dict(q=A, k=A, v=A, o=A, do=A, lse=A, dq=A, dk=A, dv=A, B=1, H=1, Nq=128, Nk=128, D=64, scale=0.125,
+                 causal=0, ws=A, wsb=1 << 20, in_dtype=0, g_dtype=0)
+        a.update(kw)
+        return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"], a["B"], a["H"],
+                          a["Nq"], a["Nk"], a["D"], a["scale"], a["causal"], a["ws"], a["wsb"], None, a["in_dtype"],
+                          a["g_dtype"])
+    assert bwd(do=None) == fa.FA_ERR_NULL
+    assert bwd(dv=None) == fa.FA_ERR_NULL
+    assert bwd(in_dtype=2) == fa.FA_ERR_DTYPE
+    assert bwd(g_dtype=1) == fa.FA_ERR_DTYPE
+    assert bwd(D=96) == fa.FA_ERR_HEADDIM
+    assert bwd(Nk=0) == fa.FA_ERR_SHAPE
+    assert bwd(scale=-1.0) == fa.FA_ERR_SHAPE
+    assert bwd(dk=A + 8) == fa.FA_ERR_ALIGN
+    assert bwd(ws=None) == fa.FA_ERR_WORKSPACE
+    assert bwd(wsb=fa.fa_bwd_workspace_bytes(1, 1, 128) - 1) == fa.FA_ERR_WORKSPACE
+    assert fa.fa_bwd_workspace_bytes(2, 3, 100) == 2560  # 2*3*100*4 = 2400 rounded up to 256
+
+
 def test_device_status_null(lib):
     assert lib.fa_device_status(None, 0) == fa.FA_ERR_NULL
 
@@ -163,6 +184,7 @@ def test_no_device_is_reported(lib):
     assert _fwd(lib) == fa.FA_ERR_DEVICE
     assert lib.fa_fwd_prefix(A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 10, None, None, 0, 0) == fa.FA_ERR_DEVICE
     assert _dec(lib) == fa.FA_ERR_DEVICE
+    assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 0, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     out = ctypes.c_int(0)
     assert lib.fa_device_status(ctypes.byref(out), 0) == fa.FA_ERR_DEVICE
