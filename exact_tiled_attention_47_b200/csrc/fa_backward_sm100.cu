@@ -65,7 +65,8 @@ struct BwdParams {
 
 struct BwdBars {
   uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
-  uint64_t st_full[kStages], st_empty[kStages];  // streamed tiles (K + V, or Q + dO + row stats)
+  uint64_t st_full[kStages], st_empty[kStages];  // streamed tiles (K + V, or Q + dO)
+  uint64_t stat_full[kStages];                   // dK/dV: the streamed block's LSE and Drow in shared memory
   uint64_t s_full, p_full, o_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -161,6 +162,7 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->st_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
+      mbar_init(&bars->stat_full[s], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, 4);
@@ -397,23 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int jj = 0; jj < n; ++jj) {
       const int i = i_first + jj, st = jj % kStages;
       if (!(ok = warp_wait(&bars->st_empty[st], ((jj / kStages) & 1) ^ 1, abort_flag, p.status))) break;
-      // the block's LSE (log2 units; +inf for rows without keys or past the end, so P = 0) and Drow
-      float* stat = sStat + st * 2 * kBT;
-      const size_t base = (static_cast<size_t>(b) * p.H + h) * Lq;
-      for (int c = lane; c < kBT; c += 32) {
-        const int qi = i * kBT + c;
-        float l2 = INFINITY, dr = 0.f;
-        if (qi < Lq) {
-          const float lse = p.lse[base + qi];
-          if (lse != -INFINITY) l2 = lse * kLog2e;
-          dr = p.drow[base + qi];
-        }
-        stat[c] = l2;
-        stat[kBT + c] = dr;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);  // release orders the stores above
+      if (lane == 0) {  // the tiles first, so their copies overlap the loads of the row statistics
+        mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
           tma_load_3d_hint(&tm_q, &bars->st_full[st], sQ(st) + pn * kPanelBytes, pn * 64, h, b * Lq + i * kBT, keep);
@@ -421,6 +408,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       issued = jj + 1;
+      // the block's LSE (log2 units; +inf for rows without keys or past the end, so P = 0) and Drow:
+      // all eight loads of a lane are independent and in flight together
+      float* stat = sStat + st * 2 * kBT;
+      const size_t base = (static_cast<size_t>(b) * p.H + h) * Lq;
+      float lv[4], dv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int qi = i * kBT + lane + 32 * u;
+        const bool in = qi < Lq;
+        lv[u] = in ? p.lse[base + qi] : -INFINITY;
+        dv[u] = in ? p.drow[base + qi] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        stat[lane + 32 * u] = (lv[u] != -INFINITY) ? lv[u] * kLog2e : INFINITY;
+        stat[kBT + lane + 32 * u] = dv[u];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->stat_full[st]);  // release: orders the warp's stores above
     }
     if (!ok && lane == 0) {
       drain_wait(&bars->fixed_full, 0);
@@ -458,9 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int jj = 0; jj < n; ++jj) {
       const int i = i_first + jj, st = jj % kStages;
       if (!(ok = warp_wait(&bars->s_full, jj & 1, abort_flag, p.status))) break;
-      // the stage's LSE/Drow: the producer stored them before its arrival on st_full (already
-      // complete here; this stage cannot be refilled before this block's P V products)
-      if (!(ok = warp_wait(&bars->st_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
+      // the stage's LSE/Drow (this stage cannot be refilled before this block's P V products)
+      if (!(ok = warp_wait(&bars->stat_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
       tc_fence_after();
       const float* stat = sStat + st * 2 * kBT;
       // key kj is visible to query q iff q >= kj - diag (causal); whole block visible iff its first
