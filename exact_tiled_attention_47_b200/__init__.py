@@ -19,7 +19,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 
 __all__ = [
     "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
-    "fa_device_status", "fa_abi_version", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
+    "fa_device_status", "fa_abi_version", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
 
@@ -167,6 +167,13 @@ def fa_device_status(clear: bool = True) -> int:
     if st != FA_OK:
         raise FAError(st, "fa_device_status")
     return out.value
+
+
+def fa_selftest_wait_timeout(stream=None):
+    """Run the bounded-wait self-test; returns (status, waited_ms)."""
+    w = ctypes.c_int(0)
+    st = load().fa_selftest_wait_timeout(ctypes.byref(w), _stream(stream))
+    return int(st), int(w.value)
 
 
 def fa_abi_version() -> int:

@@ -27,6 +27,7 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_device_status": (_I, [ctypes.POINTER(_I), _I]),
     "fa_abi_version": (_I, []),
+    "fa_selftest_wait_timeout": (_I, [ctypes.POINTER(_I), _P]),
 }
 
 _lock = threading.Lock()

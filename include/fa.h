@@ -206,6 +206,20 @@ int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_
                               int B, int H, int Nk, int D, float scale, int num_splits,
                               fa_stream_t stream, int in_dtype, int o_dtype);
 
+/*
+ * fa_selftest_wait_timeout -- run the kernels' bounded wait on a barrier that nothing arrives on.
+ *
+ * The pages describe nothing like this; it lets a caller check, on its own GPU, that a stalled wait
+ * inside this library ends with an error instead of a hang: a one-thread kernel waits with the
+ * library's bounded mbarrier wait (one second without progress), which then records FA_ERR_TIMEOUT
+ * in the device status word (see fa_device_status) and returns.  Takes about one second; the CUDA
+ * context stays usable.  *waited_ms receives the time the wait took (milliseconds), or -1 if the
+ * wait unexpectedly completed.  Synchronises `stream`; uses a mapped host word (allocates and frees
+ * it).  Returns FA_OK when the kernel ran to completion (the timeout itself is reported through the
+ * status word), FA_ERR_NULL, FA_ERR_DEVICE or FA_ERR_LAUNCH.
+ */
+int fa_selftest_wait_timeout(int* waited_ms, fa_stream_t stream);
+
 /* fa_status_string -- static English text for a status code (never NULL). */
 const char* fa_status_string(int status);
 

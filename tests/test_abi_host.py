@@ -184,6 +184,8 @@ def test_no_device_is_reported(lib):
     assert _fwd(lib) == fa.FA_ERR_DEVICE
     assert lib.fa_fwd_prefix(A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 10, None, None, 0, 0) == fa.FA_ERR_DEVICE
     assert _dec(lib) == fa.FA_ERR_DEVICE
+    w = ctypes.c_int(0)
+    assert lib.fa_selftest_wait_timeout(ctypes.byref(w), None) == fa.FA_ERR_DEVICE
     assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 0, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     out = ctypes.c_int(0)
