@@ -204,6 +204,61 @@ def timed(fn, steps, stream, dist=None):
     return ms
 
 
+def sharded_leg(args, kc, vc, dev, rank, world, dist, pk, pk_kind, fa, torch, stream, steps):
+    """Long-context decode with the cache cut along the key axis over the ranks (strong scaling).
+
+    The resident decode cache [64, 8192, 32, 128] is read as 4 sequences of 131072 keys; rank r
+    holds keys shard_range(131072, world, r) of it, runs the shard kernels, the ranks all-gather the
+    fp32 (O, LSE) blocks (no exchange with one rank), and every rank merges them.  Timing only: the
+    shards of different ranks come from each rank's own seeded cache.
+    """
+    from exact_tiled_attention_47_b200.sharded import gather_parts, part_floats, shard_range
+    g = si.CONFIGS["decode_long"]
+    B, Nk, H, D, S = g["B"], g["Nk"], g["H"], g["D"], g["num_splits"]
+    kl, vl = kc.view(B, Nk, H, D), vc.view(B, Nk, H, D)
+    off, n = shard_range(Nk, world, rank)
+    if world > 1:
+        kl = kl[:, off:off + n].contiguous()
+        vl = vl[:, off:off + n].contiguous()
+    q = to_dev(si.batched(g["seed"], si.Q_ID, B, (1, H, D), "bf16"), "bf16", dev)
+    nf = part_floats(B, H, D)
+    part = torch.empty(nf, dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_bytes(B, H, D, S), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+
+    def step():
+        st = fa.fa_decode_splitkv_shard(q, kl, vl, part, B, H, H, n, off, Nk, D, g["scale"], S, None, ws,
+                                        stream=stream)
+        if st:
+            raise fa.FAError(st, "fa_decode_splitkv_shard")
+        parts = gather_parts(part, world)
+        st = fa.fa_decode_merge(parts, world, B, H, D, o, lse, stream=stream)
+        if st:
+            raise fa.FAError(st, "fa_decode_merge")
+
+    for _ in range(args.warmup):
+        step()
+    ms = timed(step, steps, stream, dist)
+    if fa.fa_device_status(clear=True) != 0:
+        raise RuntimeError("device status set during the timed sharded decode run")
+    t = ms / steps * 1e-3
+    shard_bytes = 2 * B * n * H * D * 2
+    total_bytes = 2 * B * Nk * H * D * 2
+    gbs_rank = shard_bytes / t / 1e9
+    return {"metric": "key-sharded long-context decode HBM GB/s", "value": total_bytes / t / 1e9, "unit": "GB/s",
+            "scaling": "strong", "shards": world, "ms_per_step": ms / steps, "steps": steps,
+            "config": {"workload": "decode_long", "B": B, "H": H, "Nk_total": Nk, "Nk_shard": n, "D": D,
+                       "num_splits_per_shard": S, "dtype": "bf16",
+                       "exchange": "NCCL all-gather of fp32 (O, LSE) blocks" if world > 1 else "none (one shard)",
+                       "exchange_bytes_per_rank": 4 * nf * world if world > 1 else 0,
+                       "l2": f"K/V shard {shard_bytes / 1e9:.2f} GB vs 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs_rank / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy", "traffic": None,
+                         "algorithmic_bytes_per_step": shard_bytes},
+            "gpu_launches": 3 * steps}
+
+
 # ------------------------------------------------------------------------------------------------
 # CPU oracle legs
 
@@ -512,6 +567,8 @@ def main():
                             "frac": gbs / pk["hbm_gbs"], "traffic": measured_traffic("decode", Bd),
                             "peak_kind": f"{pk_kind} copy", "algorithmic_bytes_per_step": alg_bytes},
                "gpu_launches": 2 * dsteps}
+        if Bd == c["B"]:
+            dec["sharded"] = sharded_leg(args, kc, vc, dev, rank, world, dist, pk, pk_kind, fa, torch, stream, dsteps)
         del qd_, kc, vc, o_, l_, ws
         torch.cuda.empty_cache()
 

@@ -19,7 +19,8 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 
 __all__ = [
     "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
-    "fa_device_status", "fa_abi_version", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "attention", "decode", "FAError", "LibraryMissing",
+    "fa_device_status", "fa_abi_version", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
+    "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
 
@@ -115,6 +116,34 @@ def fa_decode_splitkv_gqa(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale,
                                      int(Hkv), int(Nk), int(D), float(scale), int(num_splits), _ptr(seqlens_k),
                                      _ptr(workspace), int(workspace_bytes), _stream(stream), int(in_dtype),
                                      int(o_dtype))
+
+
+def fa_decode_part_bytes(B, H, D) -> int:
+    return int(load().fa_decode_part_bytes(int(B), int(H), int(D)))
+
+
+def fa_decode_splitkv_shard(q, k_shard, v_shard, part, B, Hq, Hkv, Nk_shard, key_offset, Nk_total, D, scale,
+                            num_splits, seqlens_k, workspace, workspace_bytes=None, stream=None,
+                            in_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_splitkv_shard``; returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_decode_splitkv_shard(_ptr(q), _ptr(k_shard), _ptr(v_shard), _ptr(part), int(B), int(Hq),
+                                       int(Hkv), int(Nk_shard), int(key_offset), int(Nk_total), int(D),
+                                       float(scale), int(num_splits), _ptr(seqlens_k), _ptr(workspace),
+                                       int(workspace_bytes), _stream(stream), int(in_dtype))
+
+
+def fa_decode_merge(parts, R, B, H, D, o, lse, stream=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_merge``; returns its status."""
+    lib = load()
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    return lib.fa_decode_merge(_ptr(parts), int(R), int(B), int(H), int(D), _ptr(o), _ptr(lse), _stream(stream),
+                               int(o_dtype))
 
 
 def fa_decode_splitkv(q, k_cache, v_cache, o, lse, B, H, Nk, D, scale, num_splits, workspace,

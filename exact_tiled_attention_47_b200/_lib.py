@@ -24,6 +24,9 @@ SIGNATURES = {
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _Z, _P, _I, _I]),
     "fa_decode_splitkv_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _Z, _P, _I, _I]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _I, _I]),
+    "fa_decode_part_bytes": (_Z, [_I, _I, _I]),
+    "fa_decode_splitkv_shard": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _Z, _P, _I]),
+    "fa_decode_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_device_status": (_I, [ctypes.POINTER(_I), _I]),
     "fa_abi_version": (_I, []),

@@ -169,13 +169,16 @@ namespace {
 
 int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
                 int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k, void* workspace,
-                size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype) {
+                size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype, int key_offset = 0,
+                int Nk_total = 0) {
   if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_NULL;
   if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
   if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
   if (D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || Nk < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_SHAPE;
+  if (Nk_total == 0) Nk_total = Nk;
+  if (key_offset < 0 || static_cast<int64_t>(key_offset) + Nk > Nk_total) return FA_ERR_SHAPE;
   if (num_splits < 1 || num_splits > 128) return FA_ERR_SHAPE;
   if (static_cast<int64_t>(B) * H > (static_cast<int64_t>(1) << 28)) return FA_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
@@ -208,6 +211,8 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o
   a.o_fp32 = o_dtype == FA_FP32;
   a.Hkv = Hkv;
   a.seqlens_k = seqlens_k;
+  a.key_offset = key_offset;
+  a.Nk_total = Nk_total;
   const int e = fa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != 0) {
     cudaGetLastError();
@@ -233,6 +238,51 @@ int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cach
                           int o_dtype) {
   return decode_impl(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k, workspace,
                      workspace_bytes, stream, in_dtype, o_dtype);
+}
+
+size_t fa_decode_part_bytes(int B, int H, int D) {
+  if (B < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+  const size_t bytes = static_cast<size_t>(B) * H * (D + 1) * sizeof(float);
+  return (bytes + 15) & ~static_cast<size_t>(15);
+}
+
+int fa_decode_splitkv_shard(const void* q, const void* k_shard, const void* v_shard, float* part, int B,
+                            int Hq, int Hkv, int Nk_shard, int key_offset, int Nk_total, int D, float scale,
+                            int num_splits, const int* seqlens_k, void* workspace, size_t workspace_bytes,
+                            fa_stream_t stream, int in_dtype) {
+  if (!part) return FA_ERR_NULL;
+  if (Nk_total < 1) return FA_ERR_SHAPE;
+  float* lse = (B >= 1 && Hq >= 1 && (D == 64 || D == 128)) ? part + static_cast<size_t>(B) * Hq * D : part;
+  return decode_impl(q, k_shard, v_shard, part, lse, B, Hq, Hkv, Nk_shard, D, scale, num_splits, seqlens_k,
+                     workspace, workspace_bytes, stream, in_dtype, FA_FP32, key_offset, Nk_total);
+}
+
+int fa_decode_merge(const float* parts, int R, int B, int H, int D, void* o, float* lse, fa_stream_t stream,
+                    int o_dtype) {
+  if (!parts || !o || !lse) return FA_ERR_NULL;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP16 && o_dtype != FA_FP32) return FA_ERR_DTYPE;
+  if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (R < 1 || R > 65536 || B < 1 || H < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * H > (static_cast<int64_t>(1) << 28)) return FA_ERR_SHAPE;
+  if (!fa::aligned(parts, 16) || !fa::aligned(o, 16) || !fa::aligned(lse, 4)) return FA_ERR_ALIGN;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  fa::MergeArgs a;
+  a.parts = parts;
+  a.part_floats = static_cast<long long>(fa_decode_part_bytes(B, H, D) / sizeof(float));
+  a.R = R;
+  a.B = B;
+  a.H = H;
+  a.D = D;
+  a.o = o;
+  a.lse = lse;
+  a.o_fp16 = o_dtype == FA_FP16;
+  a.o_fp32 = o_dtype == FA_FP32;
+  if (fa::launch_decode_merge(a, reinterpret_cast<cudaStream_t>(stream)) != 0) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 int fa_device_status(int* status_out, int clear) {

@@ -16,6 +16,12 @@
 //   w_s = exp(lse_s - M), O = sum_s w_s o_s / sum_s w_s, LSE = M + ln sum_s w_s -- the pairwise
 //   merge of group statistics of "轻松读懂FlashAttention 上" ("Softmax求解重构") applied to all
 //   splits at once; a query without any key (valid length 0) gets O = 0, LSE = -inf.
+//
+// Key-sharded decode (a cache too long for one GPU cut along the key axis): kernel 1 runs on one
+// shard, seeing the shard's rows as keys [key_offset, key_offset + Nk) of the whole cache, and
+// kernel 2 leaves that shard's fp32 (O, LSE).  The same combine kernel, with other strides, then
+// merges the R shards' results gathered from all ranks (launch_decode_merge): the merge is
+// associative, so combining splits first and shards second gives the softmax over all keys.
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 
@@ -38,11 +44,24 @@ struct DecParams {
   float* lse;
   float* ws_o;
   float* ws_lse;
-  const int* seqlens_k;  // nullable
+  const int* seqlens_k;  // nullable; lengths of the whole cache
   int* status;
-  int B, H, Nk, S;  // H: query heads
+  int B, H, Nk, S;  // H: query heads; Nk: cache rows held here
   int Hkv, group;   // KV heads; query heads per KV head (H = Hkv * group)
+  int key_offset;   // first key of the whole cache held here
+  int Nk_total;     // keys of the whole cache
   float scale_log2;
+};
+
+// Partial results to merge: partial t of output row r (= b * H + h) has its normalised output at
+// po + r * o_row + t * o_part (D floats) and its natural-log LSE at pl + r * l_row + t * l_part.
+struct CombParams {
+  const float* po;
+  const float* pl;
+  long long o_row, o_part, l_row, l_part;
+  int T, rows;
+  void* o;
+  float* lse;
 };
 
 template <bool kFp16>
@@ -69,14 +88,15 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = lane % LPK, kk = lane / LPK;
 
-  int len = p.Nk;
+  int len = p.Nk_total;
   if (p.seqlens_k != nullptr) {
     len = __ldg(p.seqlens_k + b);
-    if (len < 0 || len > p.Nk) {  // reported, and the batch item is treated as having no keys
+    if (len < 0 || len > p.Nk_total) {  // reported, and the batch item is treated as having no keys
       if (tid == 0 && s == 0 && blockIdx.x == 0) record_status(p.status, kStatusCuSeqlens);
       len = 0;
     }
   }
+  len = min(max(len - p.key_offset, 0), p.Nk);  // valid keys among the rows held here
   const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
   const int lo = min(len, s * per);
   const int hi = min(len, lo + per);
@@ -225,21 +245,21 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 }
 
 template <bool kFp16, int D, bool kOutF32>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecParams p) {
+__global__ void __launch_bounds__(128) decode_combine_kernel(const CombParams p) {
   constexpr int PER = D / 32;  // output elements per lane
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (bh >= p.B * p.H) return;
-  const float* wl = p.ws_lse + static_cast<size_t>(bh) * p.S;
-  const float* wo = p.ws_o + static_cast<size_t>(bh) * p.S * D;
+  if (bh >= p.rows) return;
+  const float* wl = p.pl + static_cast<long long>(bh) * p.l_row;
+  const float* wo = p.po + static_cast<long long>(bh) * p.o_row;
 
   float mx = -INFINITY;
-  for (int s = lane; s < p.S; s += 32) mx = fmaxf(mx, wl[s] * kLog2e);
+  for (int t = lane; t < p.T; t += 32) mx = fmaxf(mx, wl[t * p.l_part] * kLog2e);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const bool empty = (mx == -INFINITY);  // no split saw a key (warp-uniform)
+  const bool empty = (mx == -INFINITY);  // no partial saw a key (warp-uniform)
   float wsum = 0.f;
-  for (int s = lane; s < p.S; s += 32) wsum += ex2(wl[s] * kLog2e - mx);
+  for (int t = lane; t < p.T; t += 32) wsum += ex2(wl[t * p.l_part] * kLog2e - mx);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
   const float inv = empty ? 0.f : 1.f / wsum;
@@ -247,9 +267,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecParams p) 
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int s = 0; s < p.S && !empty; ++s) {
-    const float w = ex2(wl[s] * kLog2e - mx) * inv;
-    const float* row = wo + static_cast<size_t>(s) * D + lane * PER;
+  for (int t = 0; t < p.T && !empty; ++t) {
+    const float w = ex2(wl[t * p.l_part] * kLog2e - mx) * inv;
+    const float* row = wo + t * p.o_part + lane * PER;
     if constexpr (PER == 4) {
       const float4 x = *reinterpret_cast<const float4*>(row);
       acc[0] = fmaf(w, x.x, acc[0]); acc[1] = fmaf(w, x.y, acc[1]);
@@ -284,18 +304,33 @@ void launch_split(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) 
 }
 
 template <bool kFp16, int D>
+void launch_combine(const CombParams& c, bool o_fp32, cudaStream_t stream) {
+  const dim3 cgrid((c.rows + 3) / 4);
+  if (o_fp32)
+    decode_combine_kernel<kFp16, D, true><<<cgrid, 128, 0, stream>>>(c);
+  else
+    decode_combine_kernel<kFp16, D, false><<<cgrid, 128, 0, stream>>>(c);
+}
+
+template <bool kFp16, int D>
 int launch_decode_t(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
   // query heads per CTA: the largest of 8, 4, 2, 1 that divides the group
   if (p.group % 8 == 0) launch_split<kFp16, D, 8>(a, p, stream);
   else if (p.group % 4 == 0) launch_split<kFp16, D, 4>(a, p, stream);
   else if (p.group % 2 == 0) launch_split<kFp16, D, 2>(a, p, stream);
   else launch_split<kFp16, D, 1>(a, p, stream);
-  const int nbh = a.B * a.H;
-  const dim3 cgrid((nbh + 3) / 4);
-  if (a.o_fp32)
-    decode_combine_kernel<kFp16, D, true><<<cgrid, 128, 0, stream>>>(p);
-  else
-    decode_combine_kernel<kFp16, D, false><<<cgrid, 128, 0, stream>>>(p);
+  CombParams c;
+  c.po = p.ws_o;
+  c.pl = p.ws_lse;
+  c.o_row = static_cast<long long>(p.S) * D;
+  c.o_part = D;
+  c.l_row = p.S;
+  c.l_part = 1;
+  c.T = p.S;
+  c.rows = a.B * a.H;
+  c.o = p.o;
+  c.lse = p.lse;
+  launch_combine<kFp16, D>(c, a.o_fp32, stream);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -310,9 +345,34 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.B = a.B; p.H = a.H; p.Nk = a.Nk; p.S = a.S;
   p.Hkv = a.Hkv > 0 ? a.Hkv : a.H;
   p.group = a.H / p.Hkv;
+  p.key_offset = a.key_offset;
+  p.Nk_total = a.Nk_total > 0 ? a.Nk_total : a.Nk;
   p.scale_log2 = a.scale * kLog2e;
   if (a.D == 64) return a.fp16 ? launch_decode_t<true, 64>(a, p, stream) : launch_decode_t<false, 64>(a, p, stream);
   return a.fp16 ? launch_decode_t<true, 128>(a, p, stream) : launch_decode_t<false, 128>(a, p, stream);
+}
+
+int launch_decode_merge(const MergeArgs& a, cudaStream_t stream) {
+  CombParams c;
+  const long long rows = static_cast<long long>(a.B) * a.H;
+  c.po = a.parts;
+  c.pl = a.parts + rows * a.D;
+  c.o_row = a.D;
+  c.o_part = a.part_floats;
+  c.l_row = 1;
+  c.l_part = a.part_floats;
+  c.T = a.R;
+  c.rows = static_cast<int>(rows);
+  c.o = a.o;
+  c.lse = a.lse;
+  if (a.D == 64) {
+    if (a.o_fp16) launch_combine<true, 64>(c, a.o_fp32, stream);
+    else launch_combine<false, 64>(c, a.o_fp32, stream);
+  } else {
+    if (a.o_fp16) launch_combine<true, 128>(c, a.o_fp32, stream);
+    else launch_combine<false, 128>(c, a.o_fp32, stream);
+  }
+  return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace fa

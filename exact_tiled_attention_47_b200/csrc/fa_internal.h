@@ -38,6 +38,22 @@ struct DecodeArgs {
   int o_fp32;
   int Hkv = 0;                     // KV heads (0: same as H); H is a multiple of it
   const int* seqlens_k = nullptr;  // device int32[B]: valid cache length per batch item (nullptr: Nk)
+  // The cache may be one key shard of a longer cache: its rows are the keys [key_offset,
+  // key_offset + Nk) of a cache of Nk_total keys (0: Nk), and seqlens_k counts keys of the whole cache.
+  int key_offset = 0;
+  int Nk_total = 0;
+};
+
+// Merge of R partial decode results (one per key shard) laid out as R packed blocks of part_floats
+// floats: block r holds O_r [B, H, D] then LSE_r [B, H].
+struct MergeArgs {
+  const float* parts;
+  long long part_floats;
+  int R, B, H, D;
+  void* o;
+  float* lse;
+  int o_fp16;  // 16-bit output: fp16 (1) or bf16 (0); ignored with o_fp32
+  int o_fp32;
 };
 
 struct BackwardArgs {
@@ -62,6 +78,7 @@ struct BackwardArgs {
 // Return a cudaError_t-compatible code (0 = success).
 int launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int launch_decode_merge(const MergeArgs& a, cudaStream_t stream);
 int launch_backward(const BackwardArgs& a, cudaStream_t stream);
 
 int* device_status_ptr();  // address of this device's status word (nullptr on failure)

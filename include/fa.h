@@ -184,6 +184,58 @@ int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cach
                           fa_stream_t stream, int in_dtype, int o_dtype);
 
 /*
+ * fa_decode_part_bytes -- size of one key shard's partial decode result (see
+ * fa_decode_splitkv_shard): O [B, H, D] fp32 followed by LSE [B, H] fp32, padded to a multiple of
+ * 16 bytes.  R shards' results laid end to end at this stride form the input of fa_decode_merge.
+ * Returns 0 for invalid arguments.
+ */
+size_t fa_decode_part_bytes(int B, int H, int D);
+
+/*
+ * fa_decode_splitkv_shard -- single-token decode over ONE key shard of a cache cut along the key
+ * axis (one shard per GPU), leaving the shard's partial result for fa_decode_merge.
+ *
+ * Passage: "轻松读懂FlashAttention 上", section "内存卡点" (contexts of 64k to 128k tokens and more,
+ * far beyond on-chip memory), and the merge of per-group softmax statistics of its section
+ * "Softmax求解重构": a shard's normalised output and LSE are the statistics of one key group, so
+ * the merge of all shards' results is the softmax over the whole cache.
+ *
+ * The shard holds keys [key_offset, key_offset + Nk_shard) of a cache of Nk_total keys:
+ * k_shard, v_shard [B, Nk_shard, Hkv, D] (row j is key key_offset + j).  q [B, 1, Hq, D].
+ * seqlens_k: device int32[B] or NULL, valid lengths of the WHOLE cache (NULL: Nk_total); the shard
+ * attends to its keys below seqlens_k[b].  A length outside [0, Nk_total] is detected on the device,
+ * treated as 0, and sets the device status to FA_ERR_CU_SEQLENS.  Requires 0 <= key_offset and
+ * key_offset + Nk_shard <= Nk_total (else FA_ERR_SHAPE).
+ * part: device buffer of fa_decode_part_bytes(B, Hq, D) bytes, 16-byte aligned, owned by the
+ * caller; receives the shard's fp32 O (normalised over the shard's keys; 0 where it has none) and
+ * natural-log LSE (-inf where it has none).  The split-KV kernels of fa_decode_splitkv_gqa run on
+ * the shard with `workspace` (at least fa_decode_workspace_bytes(B, Hq, D, num_splits) bytes).
+ * Other arguments, limits and errors as fa_decode_splitkv_gqa.
+ */
+int fa_decode_splitkv_shard(const void* q, const void* k_shard, const void* v_shard, float* part, int B,
+                            int Hq, int Hkv, int Nk_shard, int key_offset, int Nk_total, int D, float scale,
+                            int num_splits, const int* seqlens_k, void* workspace, size_t workspace_bytes,
+                            fa_stream_t stream, int in_dtype);
+
+/*
+ * fa_decode_merge -- merge R key shards' partial decode results into the output of the whole cache.
+ *
+ * Passage: "轻松读懂FlashAttention 上", section "Softmax求解重构" (merge of group statistics),
+ * applied to R groups at once: with M = max_r LSE_r and w_r = exp(LSE_r - M),
+ * O = sum_r w_r O_r / sum_r w_r and LSE = M + ln sum_r w_r; a row with LSE_r = -inf in every shard
+ * gets O = 0, LSE = -inf.
+ *
+ * parts: device fp32, R blocks of fa_decode_part_bytes(B, H, D) bytes each (block r as written by
+ * fa_decode_splitkv_shard for shard r, e.g. gathered from R ranks), 16-byte aligned.  The order of
+ * the blocks does not matter.  o [B, 1, H, D] of o_dtype (FA_BF16, FA_FP16 or FA_FP32), 16-byte
+ * aligned; lse [B, H] fp32.  1 <= R <= 65536.  One kernel on `stream`; nothing is allocated.
+ * Errors: FA_ERR_NULL, FA_ERR_DTYPE (o_dtype), FA_ERR_HEADDIM, FA_ERR_SHAPE, FA_ERR_ALIGN,
+ * FA_ERR_DEVICE, FA_ERR_LAUNCH.
+ */
+int fa_decode_merge(const float* parts, int R, int B, int H, int D, void* o, float* lse, fa_stream_t stream,
+                    int o_dtype);
+
+/*
  * fa_decode_splitkv_noalloc -- fa_decode_splitkv without a caller-provided workspace.
  *
  * The pages describe nothing like this; it exists for callers that cannot allocate device memory

@@ -8,7 +8,7 @@ library.  The two sides share only the seeded input generator, which holds no at
 Modules:
   attention  -- the materialised definition O = softmax(scale*Q*K^T + mask)*V with LSE, per (b, h);
                 dense, packed-varlen, row-sampled and single-query (decode) forms, the latter also
-                with grouped KV heads and per-sequence cache lengths.
+                with grouped KV heads, per-sequence cache lengths and over one key shard of a cache.
   online     -- the tiled algorithm in the order the pages give it (Q blocks outside, K/V blocks
                 inside, running max m and running sum l), and the pairwise merge of softmax
                 statistics of key groups, including the split-KV partial/combine form.
@@ -16,7 +16,8 @@ Modules:
   backward   -- dQ, dK, dV: the derivative of the forward definition for an upstream gradient dO.
 """
 from .attention import (attention_head, attention_dense, attention_varlen, attention_rows,
-                        attention_decode, attention_decode_gqa, padded_key_mask_attention)
+                        attention_decode, attention_decode_gqa, attention_decode_shard,
+                        padded_key_mask_attention)
 from .online import (tiled_online_attention, group_stats, merge_groups, softmax_by_groups,
                      split_kv_partials, combine_partials)
 from .brute import brute_attention_head
@@ -24,7 +25,7 @@ from .backward import attention_head_backward, attention_dense_backward, backwar
 
 __all__ = [
     "attention_head", "attention_dense", "attention_varlen", "attention_rows", "attention_decode",
-    "attention_decode_gqa",
+    "attention_decode_gqa", "attention_decode_shard",
     "padded_key_mask_attention", "tiled_online_attention", "group_stats", "merge_groups",
     "softmax_by_groups", "split_kv_partials", "combine_partials", "brute_attention_head",
     "attention_head_backward", "attention_dense_backward", "backward_row_terms",

@@ -196,3 +196,20 @@ def attention_decode_gqa(q, k_cache, v_cache, scale: float, seqlens_k=None):
             o[b, :, h, :], lse[b, h] = ob, lb[0]
     return o, lse
 
+
+
+def attention_decode_shard(q, k_shard, v_shard, scale: float, key_offset: int, seqlens_k=None):
+    """Decode over one key shard of a longer cache: O [B,1,Hq,Dv] and LSE [B,Hq] of the shard alone.
+
+    k_shard/v_shard [B,Nk_shard,Hkv,D] hold keys [key_offset, key_offset + Nk_shard) of the whole
+    cache; ``seqlens_k`` (optional) counts valid keys of the whole cache, so the shard sees its keys
+    below seqlens_k[b].  The result is the definition restricted to those keys (O = 0, LSE = -inf
+    where there are none): the softmax statistics of one key group in the sense of
+    "轻松读懂FlashAttention 上", section "Softmax求解重构", which merge into the whole cache's
+    result.
+    """
+    nk = k_shard.shape[1]
+    lens = None
+    if seqlens_k is not None:
+        lens = [min(max(int(L) - key_offset, 0), nk) for L in seqlens_k]
+    return attention_decode_gqa(q, k_shard, v_shard, scale, lens)

@@ -42,6 +42,11 @@ CONFIGS = {
     # grouped KV heads (4 query heads per KV head) and per-sequence cache lengths U{1024..8192}
     "decode_gqa": dict(B=64, Nk=8192, H=32, Hkv=8, D=128, dtype="bf16", scale=1.0 / math.sqrt(128),
                        num_splits=16, seed=6, len_lo=1024, len_hi=8192),
+    # long-context decode, cut along the key axis over the ranks: the "decode" cache read as 4
+    # sequences of 131072 keys (sequence b is batch items 16b .. 16b+15 of "decode" laid end to end,
+    # the same bytes), with its own queries; splits are per key shard
+    "decode_long": dict(B=4, Nk=131072, H=32, D=128, dtype="bf16", scale=1.0 / math.sqrt(128),
+                        num_splits=64, seed=7, cache_of="decode"),
 }
 
 

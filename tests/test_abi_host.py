@@ -153,6 +153,45 @@ def test_decode_gqa_validation_codes(lib):
     assert gqa(wsb=need - 1) == fa.FA_ERR_WORKSPACE
 
 
+def _shard(lib, part=A, q=A, Nk=64, off=0, tot=128, sl=None, ws=A, wsb=1 << 20, in_dtype=0):
+    return lib.fa_decode_splitkv_shard(q, A, A, part, 2, 8, 2, Nk, off, tot, 128, 0.1, 4, sl, ws, wsb, None, in_dtype)
+
+
+def _merge(lib, parts=A, R=2, B=2, H=8, D=128, o=A, lse=A, o_dtype=0):
+    return lib.fa_decode_merge(parts, R, B, H, D, o, lse, None, o_dtype)
+
+
+def test_decode_shard_and_merge_validation_codes(lib):
+    assert _shard(lib, part=None) == fa.FA_ERR_NULL
+    assert _shard(lib, q=None) == fa.FA_ERR_NULL
+    assert _shard(lib, off=-1) == fa.FA_ERR_SHAPE
+    assert _shard(lib, off=65) == fa.FA_ERR_SHAPE        # keys 65..128 run past a 128-key cache
+    assert _shard(lib, tot=0) == fa.FA_ERR_SHAPE
+    assert _shard(lib, Nk=0) == fa.FA_ERR_SHAPE
+    assert _shard(lib, in_dtype=2) == fa.FA_ERR_DTYPE
+    assert _shard(lib, part=A + 4) == fa.FA_ERR_ALIGN
+    assert _shard(lib, sl=A + 2) == fa.FA_ERR_ALIGN
+    assert _shard(lib, wsb=fa.fa_decode_workspace_bytes(2, 8, 128, 4) - 1) == fa.FA_ERR_WORKSPACE
+    assert _merge(lib, parts=None) == fa.FA_ERR_NULL
+    assert _merge(lib, lse=None) == fa.FA_ERR_NULL
+    assert _merge(lib, o_dtype=3) == fa.FA_ERR_DTYPE
+    assert _merge(lib, D=96) == fa.FA_ERR_HEADDIM
+    assert _merge(lib, R=0) == fa.FA_ERR_SHAPE
+    assert _merge(lib, B=0) == fa.FA_ERR_SHAPE
+    assert _merge(lib, parts=A + 8) == fa.FA_ERR_ALIGN
+    assert _merge(lib, o=A + 2) == fa.FA_ERR_ALIGN
+
+
+def test_decode_part_bytes(lib):
+    from exact_tiled_attention_47_b200.sharded import part_floats
+    assert fa.fa_decode_part_bytes(2, 8, 128) == 2 * 8 * 129 * 4
+    assert fa.fa_decode_part_bytes(3, 1, 64) == 784             # 3 * 65 * 4 = 780, padded to 16 bytes
+    for B, H, D in ((2, 8, 128), (3, 1, 64), (7, 5, 64), (64, 32, 128)):
+        assert fa.fa_decode_part_bytes(B, H, D) == 4 * part_floats(B, H, D)
+    assert fa.fa_decode_part_bytes(0, 8, 128) == 0
+    assert fa.fa_decode_part_bytes(2, 8, 96) == 0
+
+
 def test_bwd_validation_codes(lib):
     def bwd(**kw):
         a = dict(q=A, k=A, v=A, o=A, do=A, lse=A, dq=A, dk=A, dv=A, B=1, H=1, Nq=128, Nk=128, D=64, scale=0.125,
@@ -188,6 +227,10 @@ def test_no_device_is_reported(lib):
     assert lib.fa_selftest_wait_timeout(ctypes.byref(w), None) == fa.FA_ERR_DEVICE
     assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 0, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
+    assert _shard(lib) == fa.FA_ERR_DEVICE
+    assert _shard(lib, off=64, sl=A) == fa.FA_ERR_DEVICE
+    assert _merge(lib) == fa.FA_ERR_DEVICE
+    assert _merge(lib, o_dtype=2) == fa.FA_ERR_DEVICE
     out = ctypes.c_int(0)
     assert lib.fa_device_status(ctypes.byref(out), 0) == fa.FA_ERR_DEVICE
 

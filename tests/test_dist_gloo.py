@@ -64,3 +64,82 @@ def test_single_process_defaults():
     assert bench.max_over_ranks(3.5, None) == 3.5
     assert bench.rank_seed(5, 0) == 5
     assert bench.whole_job_rate(10.0, 1000.0, 1) == pytest.approx(10.0)
+
+
+def _shard_worker(rank, world, port, out):
+    """One rank of the key-sharded decode exchange: the shard result comes from the oracle (the
+    stand-in for the shard kernel on a CPU), is packed in the library's block layout and gathered
+    with the library's exchange step; the merge of the gathered blocks must equal the decode over
+    the whole cache."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import seeded_inputs as si
+        from exact_tiled_attention_47_b200.sharded import gather_parts, part_floats, shard_range
+        B, Hq, Hkv, Nk, D, scale = 3, 4, 2, 37, 64, 0.125
+        lens = [37, 18, 0]  # the second ends inside shard 0 of 2 (keys 0..18), the third is empty
+        qb, kb, vb = si.decode_gqa_inputs(41, B, Nk, Hq, Hkv, D, "bf16")
+        q, k, v = (si.bits_to_float(t, "bf16") for t in (qb, kb, vb))
+        off, n = shard_range(Nk, world, rank)
+        o_r, l_r = oracle.attention_decode_shard(q, k[:, off:off + n], v[:, off:off + n], scale, off, lens)
+        nf = part_floats(B, Hq, D)
+        part = torch.full((nf,), float("nan"), dtype=torch.float32)
+        part[:B * Hq * D] = torch.from_numpy(o_r.reshape(-1).astype(np.float32))
+        part[B * Hq * D:B * Hq * (D + 1)] = torch.from_numpy(l_r.reshape(-1).astype(np.float32))
+        gathered = gather_parts(part, world).numpy().astype(np.float64)
+        o_ref, lse_ref = oracle.attention_decode_gqa(q, k, v, scale, lens)
+        err_o = err_l = 0.0
+        for b in range(B):
+            for h in range(Hq):
+                row = b * Hq + h
+                o_parts = [gathered[r * nf + row * D:r * nf + (row + 1) * D] for r in range(world)]
+                l_parts = [gathered[r * nf + B * Hq * D + row] for r in range(world)]
+                o, lse = oracle.combine_partials(o_parts, l_parts)
+                err_o = max(err_o, float(np.abs(o - o_ref[b, 0, h]).max()))
+                if lse_ref[b, h] == -np.inf:
+                    assert lse == -np.inf
+                else:
+                    err_l = max(err_l, abs(lse - lse_ref[b, h]))
+        mine = gathered[rank * nf:rank * nf + B * Hq * D]
+        out.put((rank, (off, n), err_o, err_l, bool(np.array_equal(mine, part[:B * Hq * D].numpy()))))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_decode_exchange_gloo():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(out.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [(0, 19), (19, 18)]   # contiguous shards covering 37 keys
+    for _, _, err_o, err_l, own_block_in_place in res:
+        assert own_block_in_place                       # block r of the gather is rank r's
+        assert err_o < 1e-6 and err_l < 1e-6            # fp32 packing is the only rounding
+
+
+def test_shard_ranges_cover_the_cache():
+    from exact_tiled_attention_47_b200.sharded import shard_range
+    for total in (8, 37, 131072, 131073):
+        for world in (1, 2, 3, 8):
+            got = [shard_range(total, world, r) for r in range(world)]
+            assert got[0][0] == 0
+            assert all(a[0] + a[1] == b[0] for a, b in zip(got, got[1:]))
+            assert got[-1][0] + got[-1][1] == total
+            assert max(n for _, n in got) - min(n for _, n in got) <= 1
+    with pytest.raises(ValueError):
+        shard_range(3, 4, 0)
+    with pytest.raises(ValueError):
+        shard_range(10, 2, 2)

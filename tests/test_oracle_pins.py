@@ -24,6 +24,8 @@ wrong LSE base, a bad group merge) fails at least one of them:
   * decode with grouped KV heads and per-sequence cache lengths: equal to the dense decode over KV
     heads repeated G times, equal to decode over the truncated cache, the Q = 0 closed form, and
     the split-KV combine with empty splits;
+  * decode over key shards of a cache: the Q = 0 closed form with the shard's own visible-key
+    count, and the merge of all shards' results equal to decode over the whole cache;
   * the backward (dQ, dK, dV): central finite differences of the forward oracle, the Q = 0 closed
     forms, invariance of dQ and dV under a common key shift, and zero total dK.
 """
@@ -449,6 +451,42 @@ def test_combine_of_empty_splits():
     o_ref, lse_ref = oracle.attention_head(q[None, :], k, v, 0.4)
     np.testing.assert_allclose(o, o_ref[0], rtol=1e-12, atol=1e-14)
     assert abs(lse - lse_ref[0]) < 1e-12
+
+
+def test_shard_results_merge_to_the_whole_cache():
+    # decode over contiguous key shards, merged with the split-KV combine, equals decode over the
+    # whole cache, for lengths ending inside, at the edge of, and before a shard (and 0)
+    B, Nk, Hkv, G, D = 5, 50, 2, 2, 8
+    q = rnd((B, 1, Hkv * G, D), 151)
+    k, v = rnd((B, Nk, Hkv, D), 152), rnd((B, Nk, Hkv, D), 153)
+    lens = [50, 17, 0, 35, 20]
+    bounds = [(0, 20), (20, 35), (35, 50)]
+    shards = [oracle.attention_decode_shard(q, k[:, lo:hi], v[:, lo:hi], 0.35, lo, lens) for lo, hi in bounds]
+    o_ref, lse_ref = oracle.attention_decode_gqa(q, k, v, 0.35, lens)
+    for b in range(B):
+        for h in range(Hkv * G):
+            o, lse = oracle.combine_partials([s[0][b, 0, h] for s in shards], [s[1][b, h] for s in shards])
+            if lens[b] == 0:
+                assert np.all(o == 0) and lse == -np.inf and lse_ref[b, h] == -np.inf
+                continue
+            np.testing.assert_allclose(o, o_ref[b, 0, h], rtol=1e-12, atol=1e-14)
+            assert abs(lse - lse_ref[b, h]) < 1e-12
+
+
+def test_shard_decode_zero_query_closed_form():
+    # Q = 0: a shard's O is the mean of ITS visible value rows and its LSE is ln(#visible keys of the
+    # shard), here keys [20, 30) of the whole cache with whole-cache lengths 25, 20, 40, 30
+    B, Nk_shard, Hkv, D, off = 4, 10, 1, 8, 20
+    q = np.zeros((B, 1, 2, D))
+    k, v = rnd((B, Nk_shard, Hkv, D), 154), rnd((B, Nk_shard, Hkv, D), 155)
+    o, lse = oracle.attention_decode_shard(q, k, v, 0.5, off, [25, 20, 40, 30])
+    for b, n in enumerate([5, 0, 10, 10]):
+        for h in range(2):
+            if n == 0:
+                assert np.all(o[b, 0, h] == 0) and lse[b, h] == -np.inf
+                continue
+            np.testing.assert_allclose(o[b, 0, h], v[b, :n, 0].mean(axis=0), rtol=RTOL, atol=1e-14)
+            assert abs(lse[b, h] - math.log(n)) < 1e-13
 
 
 # ---------------------------------------------------------------------------------------------
