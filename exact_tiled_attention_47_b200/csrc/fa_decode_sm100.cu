@@ -22,7 +22,10 @@
 // kernel 2 leaves that shard's fp32 (O, LSE).  The same combine kernel, with other strides, then
 // merges the R shards' results gathered from all ranks (launch_decode_merge): the merge is
 // associative, so combining splits first and shards second gives the softmax over all keys.
+#include <atomic>
+
 #include "fa_internal.h"
+#include "fa_prefill_common.cuh"  // bounded waits, TMA map builder
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -33,8 +36,6 @@ constexpr int kChunk = 256;
 // A split covers at least this many keys: shorter caches use fewer splits (the rest exit at once),
 // since a CTA's fixed costs (query load, reductions, partial writes) outweigh streaming a few keys.
 constexpr int kMinSplitKeys = 512;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 struct DecParams {
   const void* q;
@@ -244,6 +245,323 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Grouped decode on the tensor cores (G = 2..16 query heads per KV head).
+//
+// With G query heads sharing each K/V row, the split is a small matrix product: S = Q K^T with Q the
+// G x D block of the group's queries, then O += P V.  On CUDA cores that costs G multiply-adds per
+// loaded element plus a shuffle reduction per head, which leaves the grouped decode bound by
+// instruction issue far below HBM bandwidth.  Here warp-level mma.sync m16n8k16 tiles take both
+// products (the G heads are the M rows of a 16-row tile; rows >= G are zero), so a 16-key slice of
+// K and V costs 2 * D/8 MMAs and D/4 ldmatrix per warp, and the kernel is bound by HBM again.
+// (tcgen05 needs M >= 64 rows and a TMEM round trip per block; with at most 16 live rows the
+// register-resident warp MMA is the better fit for this matrix-vector-like product.)
+//
+// CTA = (G heads of one KV head, split, batch): warp 4 streams 64-key K and V tiles of the split
+// through a ring of kMmaStages shared-memory stages with TMA (box 64 columns x 1 head x 64 rows,
+// 128-byte swizzle, no multicast); warps 0-3 each take 16 keys of every tile: S from ldmatrix'd K
+// and Q fragments held in registers, an online softmax per head row in the log2 domain with lazy
+// rescaling (O and l share a running max that is only raised when a block max exceeds it by more
+// than 2^8, which keeps P <= 2^8 and is exact after the final division), P repacked in registers as
+// the A operand, and O += P V from transposing ldmatrix of V.  The four warps' (m, l, O) are merged
+// through shared memory at the end and the split's normalised partial and LSE are written as by
+// decode_split_kernel, so the same combine follows.
+
+constexpr int kMmaTileKeys = 64;
+constexpr int kMmaThreads = 160;  // 4 MMA warps + 1 TMA warp
+constexpr int kMmaProducerWarp = 4;
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D>
+struct MmaCfg {
+  static constexpr int kPanelBytes = kMmaTileKeys * 128;     // 64 rows x 64 columns x 2 bytes
+  static constexpr int kTileBytes = kPanelBytes * (D / 64);  // one K (or V) tile
+  static constexpr int kStages = (D == 128) ? 3 : 5;         // two CTAs per SM
+  static constexpr int kStageBytes = 2 * kTileBytes;         // K then V
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;    // barriers + alignment slack
+};
+
+struct MmaBars {
+  uint64_t full[8];
+  uint64_t empty[8];
+  int abort_flag;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+// D[16x8] += A[16x16] * B[16x8], fp32 accumulate; A and B of the same 16-bit type.
+template <bool kFp16>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (kFp16) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// Byte offset of 16-bit element (row, col) in a tile of 64-column panels of kMmaTileKeys rows with
+// the 128-byte swizzle TMA writes (16-byte chunk index XOR row % 8); col is a multiple of 8.
+__device__ __forceinline__ uint32_t swz_off(int row, int col) {
+  return static_cast<uint32_t>((col >> 6) * (kMmaTileKeys * 128) + row * 128 +
+                               ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+template <bool kFp16, int D, int G>
+__global__ void __launch_bounds__(kMmaThreads, 2)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                      const DecParams p) {
+  using C = MmaCfg<D>;
+  static_assert(G >= 2 && G <= 16, "2..16 heads per CTA");
+  constexpr bool kHi = G > 8;  // rows 8..15 of the tile carry heads
+  constexpr int KS = D / 16;   // k-steps of S = Q K^T
+  constexpr int NT = D / 8;    // 8-column tiles of O
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  MmaBars* bars = reinterpret_cast<MmaBars*>(smem + C::kBarOff);
+
+  const int s = blockIdx.y, b = blockIdx.z;
+  const int subs = p.group / G;
+  const int hk = blockIdx.x / subs;
+  const int hq0 = hk * p.group + (blockIdx.x % subs) * G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  int len = p.Nk_total;
+  if (p.seqlens_k != nullptr) {
+    len = __ldg(p.seqlens_k + b);
+    if (len < 0 || len > p.Nk_total) {
+      if (tid == 0 && s == 0 && blockIdx.x == 0) record_status(p.status, kStatusCuSeqlens);
+      len = 0;
+    }
+  }
+  len = min(max(len - p.key_offset, 0), p.Nk);
+  const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
+  const int lo = min(len, s * per);
+  const int hi = min(len, lo + per);
+  auto ws_o = [&](int g) { return p.ws_o + ((static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s) * D; };
+  auto ws_l = [&](int g) { return p.ws_lse + (static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s; };
+  if (lo >= hi) {  // uniform over the CTA: empty partials
+    for (int i = tid; i < G * D; i += kMmaThreads) ws_o(i / D)[i % D] = 0.f;
+    if (tid < G) *ws_l(tid) = -INFINITY;
+    return;
+  }
+  const int n_tiles = (hi - lo + kMmaTileKeys - 1) / kMmaTileKeys;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->empty[i], 4);
+    }
+    bars->abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &bars->abort_flag;
+
+  float m_fin[2] = {-INFINITY, -INFINITY}, l_fin[2] = {0.f, 0.f};
+  float o[NT][4];
+
+  if (warp == kMmaProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      int issued = 0;
+      const int row0 = b * p.Nk + lo;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % C::kStages;
+        if (t >= C::kStages && !mbar_wait(&bars->empty[st], ((t / C::kStages) - 1) & 1, abort_flag, p.status))
+          break;
+        uint8_t* kdst = smem + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) {
+          tma_load_3d(&tmap_k, &bars->full[st], kdst + pn * C::kPanelBytes, pn * 64, hk, row0 + t * kMmaTileKeys);
+          tma_load_3d(&tmap_v, &bars->full[st], kdst + C::kTileBytes + pn * C::kPanelBytes, pn * 64, hk,
+                      row0 + t * kMmaTileKeys);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag) {  // let the copies already issued land before the stages are reused or freed
+        for (int t = max(0, issued - C::kStages); t < issued; ++t)
+          drain_wait(&bars->full[t % C::kStages], (t / C::kStages) & 1);
+      }
+    }
+  } else {
+    const int g = lane >> 2, tg = lane & 3;
+    // Q fragments (A operand, rows = heads, scaled later): a0 (g, 2tg..), a1 (g+8, 2tg..),
+    // a2 (g, 2tg+8..), a3 (g+8, 2tg+8..) of each 16-column step
+    uint32_t qa[KS][4];
+    {
+      const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
+      const size_t qrow = (static_cast<size_t>(b) * p.H + hq0) * D;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c = ks * 16 + 2 * tg;
+        qa[ks][0] = (g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c) / 2) : 0u;
+        qa[ks][2] = (g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c + 8) / 2) : 0u;
+        qa[ks][1] = (kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c) / 2) : 0u;
+        qa[ks][3] = (kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c + 8) / 2) : 0u;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    const float sl2 = p.scale_log2;
+    const int mi = lane >> 3;  // which 8x8 matrix this lane addresses in ldmatrix.x4
+
+    for (int t = 0; t < n_tiles; ++t) {
+      const int st = t % C::kStages;
+      if (!warp_wait(&bars->full[st], (t / C::kStages) & 1, abort_flag, p.status)) break;
+      const uint32_t kb = smem_addr(smem + st * C::kStageBytes);
+      const uint32_t vb = kb + C::kTileBytes;
+
+      // S = Q K^T for this warp's 16 keys: n-tile 0 = keys 0..7, n-tile 1 = keys 8..15
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int krow = warp * 16 + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kb + swz_off(krow, ks * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+          mma16816<kFp16>(sc[0], qa[ks], b0, b1);
+          mma16816<kFp16>(sc[1], qa[ks], b2, b3);
+        }
+      }
+      // keys of this thread: n-tile n, element e -> key warp*16 + 8n + 2tg + (e & 1); e < 2 row g,
+      // e >= 2 row g + 8
+      const int key0 = lo + t * kMmaTileKeys + warp * 16 + 2 * tg;
+      const bool tail = (lo + (t + 1) * kMmaTileKeys > hi);
+      uint32_t pa[4];
+#pragma unroll
+      for (int r = 0; r < (kHi ? 2 : 1); ++r) {
+        float x[4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float v = sc[n][2 * r + e] * sl2;
+            if (tail && key0 + 8 * n + e >= hi) v = -INFINITY;
+            x[2 * n + e] = v;
+          }
+        }
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        if (mx > m_run[r] + kRescaleLog2 || (m_run[r] == -INFINITY && mx > -INFINITY)) {
+          const float alpha = ex2(m_run[r] - mx);  // 0 while nothing was accumulated
+          l_run[r] *= alpha;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            o[j][2 * r] *= alpha;
+            o[j][2 * r + 1] *= alpha;
+          }
+          m_run[r] = mx;
+        }
+        float pv[4];
+        if (m_run[r] == -INFINITY) {
+          pv[0] = pv[1] = pv[2] = pv[3] = 0.f;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pv[i] = ex2(x[i] - m_run[r]);
+        }
+        l_run[r] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+        // A operand of P V: a0/a2 hold row g (keys 2tg.. of n-tiles 0/1), a1/a3 row g + 8
+        pa[r] = pack2<kFp16>(pv[0], pv[1]);
+        pa[2 + r] = pack2<kFp16>(pv[2], pv[3]);
+      }
+      if constexpr (!kHi) {
+        pa[1] = 0u;
+        pa[3] = 0u;
+      }
+      // O += P V: ldmatrix.trans gives the B fragments of two 8-column tiles per call
+      {
+        const int vrow = warp * 16 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int dt = 0; dt < NT / 2; ++dt) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vb + swz_off(vrow, dt * 16 + (mi >> 1) * 8), b0, b1, b2, b3);
+          mma16816<kFp16>(o[2 * dt], pa, b0, b1);
+          mma16816<kFp16>(o[2 * dt + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->empty[st]);
+    }
+    // row sums over the quad (each lane summed its own keys)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+      m_fin[r] = m_run[r];
+      l_fin[r] = l_run[r];
+    }
+  }
+  __syncthreads();  // every stage consumed (or drained): the ring is free for the merge
+  const bool ok = (*abort_flag == 0);
+
+  // merge of the four MMA warps: red_o[w][h][d], red_m[w][h], red_l[w][h] over the stage memory
+  float* red_o = reinterpret_cast<float*>(smem);
+  float* red_m = red_o + 4 * G * D;
+  float* red_l = red_m + 4 * G;
+  if (ok && warp < 4) {
+    const int g = lane >> 2, tg = lane & 3;
+#pragma unroll
+    for (int r = 0; r < (kHi ? 2 : 1); ++r) {
+      const int h = g + 8 * r;
+      if (h < G) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          red_o[(warp * G + h) * D + 8 * j + 2 * tg] = o[j][2 * r];
+          red_o[(warp * G + h) * D + 8 * j + 2 * tg + 1] = o[j][2 * r + 1];
+        }
+        if (tg == 0) {
+          red_m[warp * G + h] = m_fin[r];
+          red_l[warp * G + h] = l_fin[r];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (!ok) return;
+  for (int i = tid; i < G * D; i += kMmaThreads) {
+    const int h = i / D, d = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * G + h]);
+    float l = 0.f, acc = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float e = ex2(red_m[w * G + h] - M);
+        l += e * red_l[w * G + h];
+        acc += e * red_o[(w * G + h) * D + d];
+      }
+    }
+    ws_o(h)[d] = (M > -INFINITY) ? acc / l : 0.f;
+    if (d == 0) *ws_l(h) = (M > -INFINITY) ? (M + lg2(l)) * kLn2 : -INFINITY;
+  }
+}
+
 template <bool kFp16, int D, bool kOutF32>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const CombParams p) {
   constexpr int PER = D / 32;  // output elements per lane
@@ -312,13 +630,43 @@ void launch_combine(const CombParams& c, bool o_fp32, cudaStream_t stream) {
     decode_combine_kernel<kFp16, D, false><<<cgrid, 128, 0, stream>>>(c);
 }
 
+template <bool kFp16, int D, int G>
+int launch_mma(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
+  CUtensorMap mk, mv;
+  const int rows = a.B * a.Nk;
+  if (!make_tma_map(&mk, a.k, rows, p.Hkv, D, kFp16, kMmaTileKeys) ||
+      !make_tma_map(&mv, a.v, rows, p.Hkv, D, kFp16, kMmaTileKeys))
+    return static_cast<int>(cudaErrorInvalidValue);
+  auto kern = decode_mma_kernel<kFp16, D, G>;
+  // the shared-memory opt-in is a per-device attribute of the function: set it once per device
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return static_cast<int>(cudaErrorInvalidDevice);
+  if (!((configured.load(std::memory_order_acquire) >> dev) & 1u)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MmaCfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
+  }
+  kern<<<dim3(p.Hkv * (p.group / G), a.S, a.B), kMmaThreads, MmaCfg<D>::kSmemBytes, stream>>>(mk, mv, p);
+  return 0;
+}
+
 template <bool kFp16, int D>
 int launch_decode_t(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
-  // query heads per CTA: the largest of 8, 4, 2, 1 that divides the group
-  if (p.group % 8 == 0) launch_split<kFp16, D, 8>(a, p, stream);
+  // Grouped heads: the tensor-core kernel with G = the largest of 16, 8, 4, 2 dividing the group
+  // (the TMA maps index rows with 32-bit coordinates); one head per KV head: the CUDA-core kernel.
+  const bool tma_rows_ok = static_cast<long long>(a.B) * a.Nk < (1LL << 31);
+  int e = 0;
+  if (tma_rows_ok && p.group % 16 == 0) e = launch_mma<kFp16, D, 16>(a, p, stream);
+  else if (tma_rows_ok && p.group % 8 == 0) e = launch_mma<kFp16, D, 8>(a, p, stream);
+  else if (tma_rows_ok && p.group % 4 == 0) e = launch_mma<kFp16, D, 4>(a, p, stream);
+  else if (tma_rows_ok && p.group % 2 == 0) e = launch_mma<kFp16, D, 2>(a, p, stream);
+  else if (p.group % 8 == 0) launch_split<kFp16, D, 8>(a, p, stream);
   else if (p.group % 4 == 0) launch_split<kFp16, D, 4>(a, p, stream);
   else if (p.group % 2 == 0) launch_split<kFp16, D, 2>(a, p, stream);
   else launch_split<kFp16, D, 1>(a, p, stream);
+  if (e != 0) return e;
   CombParams c;
   c.po = p.ws_o;
   c.pl = p.ws_lse;

@@ -173,8 +173,9 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, v
  * head h / (Hq / Hkv).  seqlens_k: device int32[B] (4-byte aligned) or NULL; the query of batch
  * item b attends to cached keys [0, seqlens_k[b]) (all Nk when NULL).  A length of 0 gives O = 0 and
  * LSE = -inf; a length outside [0, Nk] is detected on the device, treated as 0, and sets the device
- * status to FA_ERR_CU_SEQLENS.  Each KV row is read once for all query heads of its group (up to 8
- * per CTA).  workspace: at least fa_decode_workspace_bytes(B, Hq, D, num_splits) bytes.  Other
+ * status to FA_ERR_CU_SEQLENS.  Each KV row is read once for all query heads of its group (up to 16
+ * per CTA; groups of 2 or more heads run on the tensor cores).  workspace: at least
+ * fa_decode_workspace_bytes(B, Hq, D, num_splits) bytes.  Other
  * arguments, ownership and errors as fa_decode_splitkv; with Hkv = Hq and seqlens_k = NULL the
  * result equals fa_decode_splitkv's.
  */

@@ -49,6 +49,10 @@ CASES = [
     (2, 12, 2, 300, 64, "bf16", 16, "fp32", [5, 299]),                 # group 6: CTAs of 2, empty splits
     (2, 8, 8, 300, 128, "bf16", 8, "fp32", [123, 0]),                  # no grouping, ragged only
     (5, 8, 2, 4099, 128, "fp16", 128, "fp16", [4099, 4098, 2048, 129, 128]),
+    (2, 16, 2, 1500, 64, "bf16", 16, "fp32", [1500, 700]),            # group 8, D = 64
+    (3, 32, 4, 2000, 128, "fp16", 8, "fp32", [2000, 63, 64]),          # group 8; one partial tile
+    (4, 4, 1, 700, 64, "fp16", 2, "fp16", [65, 128, 129, 700]),       # group 4 at tile edges
+    (2, 32, 2, 1000, 64, "bf16", 4, "fp32", [1000, 511]),             # group 16, D = 64
 ]
 
 
