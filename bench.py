@@ -254,7 +254,10 @@ def sharded_leg(args, kc, vc, dev, rank, world, dist, pk, pk_kind, fa, torch, st
                        "exchange_bytes_per_rank": 4 * nf * world if world > 1 else 0,
                        "l2": f"K/V shard {shard_bytes / 1e9:.2f} GB vs 126 MB L2"},
             "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs_rank / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy", "traffic": None,
+                         "frac": gbs_rank / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy",
+                         # the same split kernel streams the same cache bytes as the plain decode: its
+                         # DRAM bytes per batch item of that cache, scaled to this rank's shard
+                         "traffic": measured_traffic("decode", shard_bytes / (2 * 8192 * H * D * 2)),
                          "algorithmic_bytes_per_step": shard_bytes},
             "gpu_launches": 3 * steps}
 
