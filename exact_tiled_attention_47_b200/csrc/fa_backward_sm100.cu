@@ -19,12 +19,17 @@
 //                       memory) and write them over S^T and dP^T, then dV += P^T dO_i and
 //                       dK += dS^T Q_i accumulate in TMEM.  dV and dK * scale are written at the end.
 // Both recompute S and dP (two more GEMMs than the minimum) so that each gradient is owned by one
-// CTA and accumulates in TMEM.  Warps 0-3 compute, warp 4 is the TMA producer, warp 5 owns TMEM and
-// issues every tcgen05.mma from one thread; the next block's S/dP are issued after the products that
-// read the previous block's P/dS columns (the tensor core runs one thread's MMAs in order).  The MMA
-// forms are those of the forward kernel: SS with both operands K-major (S, dP) and TS with the A
-// operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal runs skip fully masked
-// blocks; masking is applied on the blocks that cross the diagonal and at the sequence ends.
+// CTA and accumulates in TMEM.  Each streamed 128-row block is processed as two 64-column halves that
+// form two independent pipelines: warps 0-3 compute half 0 and warps 4-7 half 1 (the same TMEM lanes,
+// different columns), warp 8 is the TMA producer, and warp 9 owns TMEM and issues every tcgen05.mma
+// from one thread.  For each half it issues S and dP (N = 64), waits for that half's P/dS, issues the
+// half's gradient products (K = 64) and at once the next block's S and dP of the same half, so the
+// tensor core works on one half while the other half's softmax-derivative runs (the tensor core runs
+// one thread's MMAs in order, which orders each half's next S/dP after the products that read its
+// P/dS columns).  The MMA forms are those of the forward kernel: SS with both operands K-major (S, dP)
+// and TS with the A operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal runs skip
+// fully masked blocks; masking is applied on the blocks that cross the diagonal and at the sequence
+// ends.
 #include <cudaTypedefs.h>
 
 #include "fa_prefill_common.cuh"
@@ -33,9 +38,10 @@ namespace fa {
 namespace {
 
 constexpr int kBT = 128;  // rows per tile (queries or keys)
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kHalf = 64;  // columns of a half block
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr int kStages = 2;
@@ -67,7 +73,8 @@ struct BwdBars {
   uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
   uint64_t st_full[kStages], st_empty[kStages];  // streamed tiles (K + V, or Q + dO)
   uint64_t stat_full[kStages];                   // dK/dV: the streamed block's LSE and Drow in shared memory
-  uint64_t s_full, p_full, o_done, drain;
+  uint64_t s_full[2], p_full[2];                 // per half block
+  uint64_t o_done, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -122,19 +129,26 @@ __device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint32_t a, uint32_t b, 
   }
 }
 
-// d += A (TMEM, 128 x 128 packed 16-bit) * B (shared, N-major, 128 rows of D)
-__device__ __forceinline__ void mma_tn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, uint32_t idesc, bool accumulate) {
+// d += A (TMEM, 128 x 64 packed 16-bit) * B (shared, N-major, the 64 rows of a half block from b)
+__device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, uint32_t idesc,
+                                            bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < kBT / 16; ++kk)
+  for (int kk = 0; kk < kHalf / 16; ++kk)
     mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, kPanelBytes, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// Byte offset of row 64 in a 128-row swizzled tile (rows are 128 bytes in every 64-column panel).
+constexpr uint32_t kHalfRowOff = kHalf * 128;
+
 // Every lane of the warp loads (tcgen05.ld is warp-collective); only lanes with store write the row.
+// Columns [32 * ch_lo, 32 * ch_hi) of the row.
 template <int D, bool kFp16, bool kOutF32>
-__device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint32_t taddr, float mul, bool store) {
+__device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint32_t taddr, float mul, bool store,
+                                               int ch_lo = 0, int ch_hi = D / 32) {
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
+    if (ch < ch_lo || ch >= ch_hi) continue;
     uint32_t r[32];
     tmem_ld32_sync(taddr + ch * 32, r);
     if (!store) continue;
@@ -164,8 +178,10 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
       mbar_init(&bars->st_empty[s], 1);
       mbar_init(&bars->stat_full[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_full, 4);
+    for (int hh = 0; hh < 2; ++hh) {
+      mbar_init(&bars->s_full[hh], 1);
+      mbar_init(&bars->p_full[hh], 4);
+    }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -263,29 +279,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
-      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status);
+      // S = Q K_j^T and dP = dO V_j^T of half hh (keys 64 hh .. 64 hh + 63 of block j)
+      auto issue_s = [&](int st, int hh) {
+        mma_kk<D>(tbase + kColS + kHalf * hh, smem_addr(sQ), smem_addr(sK(st)) + kHalfRowOff * hh, idesc_s);
+        mma_kk<D>(tbase + kColDP + kHalf * hh, smem_addr(sDO), smem_addr(sV(st)) + kHalfRowOff * hh, idesc_s);
+        mma_commit(&bars->s_full[hh]);
+      };
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
+                mbar_wait(&bars->st_full[0], 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % kStages;
-        if (!(ok = mbar_wait(&bars->st_full[st], (j / kStages) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        mma_kk<D>(tbase + kColS, smem_addr(sQ), smem_addr(sK(st)), idesc_s);    // S = Q K_j^T
-        mma_kk<D>(tbase + kColDP, smem_addr(sDO), smem_addr(sV(st)), idesc_s);  // dP = dO V_j^T
-        mma_commit(&bars->s_full);
-        if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        mma_tn(tbase + kColA, tbase + kColDP, smem_addr(sK(st)), idesc_g, j > 0);  // dQ += dS K_j
-        mma_commit(&bars->st_empty[st]);
-        mma_commit(&bars->o_done);
+        for (int hh = 0; hh < 2; ++hh) {
+          if (!(ok = mbar_wait(&bars->p_full[hh], j & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          // dQ += dS_hh K_j[hh]
+          mma_tn_half(tbase + kColA, tbase + kColDP + kHalf * hh, smem_addr(sK(st)) + kHalfRowOff * hh, idesc_g,
+                      j > 0 || hh > 0);
+          if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
+          if (j + 1 < n) {
+            const int st1 = (j + 1) % kStages;
+            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status)))
+              break;
+            tc_fence_after();
+            issue_s(st1, hh);
+          }
+        }
       }
+      if (ok) mma_commit(&bars->o_done);
       mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int r = warp * 32 + lane;
+    const int hh = warp >> 2;  // half of every key block this warp works on
+    const int r = (warp & 3) * 32 + lane;
     const int qi = m0 + r;
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;
     const int tile_lim = p.causal ? min(Lk, m0 + 1 + diag) : Lk;
     const size_t stat = (static_cast<size_t>(b) * p.H + h) * Lq + min(qi, Lq - 1);
@@ -296,12 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      if (!(ok = warp_wait(&bars->s_full, j & 1, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(&bars->s_full[hh], j & 1, abort_flag, p.status))) break;
       tc_fence_after();
       const bool masked = (j + 1) * kBT > tile_lim;
       const int lim = row_lim - j * kBT;
 #pragma unroll
-      for (int ch = 0; ch < kBT / 32; ++ch) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int ch = 2 * hh + c2;  // 32-key chunk of the block
         uint32_t s[32], dp[32], pk[16];
         tmem_ld32_sync(lane_base + kColS + ch * 32, s);
         tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
@@ -316,18 +352,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           pk[i] = pack2<kFp16>(p0 * (__uint_as_float(dp[2 * i]) - dr), p1 * (__uint_as_float(dp[2 * i + 1]) - dr));
         }
-        tmem_st16(lane_base + kColDP + ch * 16, pk);  // dS over dP, below the unread columns
+        // dS over the half's dP, below its unread columns
+        tmem_st16(lane_base + kColDP + kHalf * hh + c2 * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[hh]);
     }
-    if (ok) ok = warp_wait(&bars->o_done, (n - 1) & 1, abort_flag, p.status);
+    if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       const size_t row = (static_cast<size_t>(b) * Lq + min(qi, Lq - 1)) * p.H + h;
-      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq);
+      // the two halves of warps store the two halves of the row
+      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, hh * D / 64,
+                                        (hh + 1) * D / 64);
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -435,35 +474,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
-      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status);
+      // S^T = K Q_i^T and dP^T = V dO_i^T of half hh (queries 64 hh .. 64 hh + 63 of block i)
+      auto issue_s = [&](int st, int hh) {
+        mma_kk<D>(tbase + kColS + kHalf * hh, smem_addr(sK), smem_addr(sQ(st)) + kHalfRowOff * hh, idesc_s);
+        mma_kk<D>(tbase + kColDP + kHalf * hh, smem_addr(sV), smem_addr(sDO(st)) + kHalfRowOff * hh, idesc_s);
+        mma_commit(&bars->s_full[hh]);
+      };
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
+                mbar_wait(&bars->st_full[0], 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
       for (int jj = 0; ok && jj < n; ++jj) {
         const int st = jj % kStages;
-        if (!(ok = mbar_wait(&bars->st_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        mma_kk<D>(tbase + kColS, smem_addr(sK), smem_addr(sQ(st)), idesc_s);    // S^T = K Q_i^T
-        mma_kk<D>(tbase + kColDP, smem_addr(sV), smem_addr(sDO(st)), idesc_s);  // dP^T = V dO_i^T
-        mma_commit(&bars->s_full);
-        if (!(ok = mbar_wait(&bars->p_full, jj & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        mma_tn(tbase + kColA, tbase + kColS, smem_addr(sDO(st)), idesc_g, jj > 0);      // dV += P^T dO_i
-        mma_tn(tbase + kColA + D, tbase + kColDP, smem_addr(sQ(st)), idesc_g, jj > 0);  // dK += dS^T Q_i
-        mma_commit(&bars->st_empty[st]);
-        mma_commit(&bars->o_done);
+        for (int hh = 0; hh < 2; ++hh) {
+          if (!(ok = mbar_wait(&bars->p_full[hh], jj & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const bool acc = jj > 0 || hh > 0;
+          // dV += P^T_hh dO_i[hh],  dK += dS^T_hh Q_i[hh]
+          mma_tn_half(tbase + kColA, tbase + kColS + kHalf * hh, smem_addr(sDO(st)) + kHalfRowOff * hh, idesc_g, acc);
+          mma_tn_half(tbase + kColA + D, tbase + kColDP + kHalf * hh, smem_addr(sQ(st)) + kHalfRowOff * hh, idesc_g,
+                      acc);
+          if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
+          if (jj + 1 < n) {
+            const int st1 = (jj + 1) % kStages;
+            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((jj + 1) / kStages) & 1, abort_flag, p.status)))
+              break;
+            tc_fence_after();
+            issue_s(st1, hh);
+          }
+        }
       }
+      if (ok) mma_commit(&bars->o_done);
       mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int r = warp * 32 + lane;
+    const int hh = warp >> 2;  // half of every query block this warp works on
+    const int r = (warp & 3) * 32 + lane;
     const int kj = n0 + r;  // this thread's key
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       const int i = i_first + jj, st = jj % kStages;
-      if (!(ok = warp_wait(&bars->s_full, jj & 1, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(&bars->s_full[hh], jj & 1, abort_flag, p.status))) break;
       // the stage's LSE/Drow (this stage cannot be refilled before this block's P V products)
       if (!(ok = warp_wait(&bars->stat_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
       tc_fence_after();
@@ -473,7 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
       const int q_lo = kj - diag - i * kBT;  // columns c < q_lo are masked
 #pragma unroll
-      for (int ch = 0; ch < kBT / 32; ++ch) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int ch = 2 * hh + c2;  // 32-query chunk of the block
         uint32_t s[32], dp[32], pk[16], dk[16];
         tmem_ld32_sync(lane_base + kColS + ch * 32, s);
         tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
@@ -496,20 +556,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           dk[2 * q4] = pack2<kFp16>(dsv[0], dsv[1]);
           dk[2 * q4 + 1] = pack2<kFp16>(dsv[2], dsv[3]);
         }
-        tmem_st16(lane_base + kColS + ch * 16, pk);   // P^T over S^T, below the unread columns
-        tmem_st16(lane_base + kColDP + ch * 16, dk);  // dS^T over dP^T
+        tmem_st16(lane_base + kColS + kHalf * hh + c2 * 16, pk);   // P^T over the half's S^T
+        tmem_st16(lane_base + kColDP + kHalf * hh + c2 * 16, dk);  // dS^T over the half's dP^T
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[hh]);
     }
-    if (ok) ok = warp_wait(&bars->o_done, (n - 1) & 1, abort_flag, p.status);
+    if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       const size_t row = ((static_cast<size_t>(b) * Lk + min(kj, Lk - 1)) * p.H + h) * D;
-      store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk);         // dV
-      store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk);  // dK
+      if (hh == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk);  // dV
+      else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk);  // dK
     }
   }
   bwd_teardown(bars, warp, tbase);
