@@ -111,6 +111,32 @@ __global__ void __launch_bounds__(256) bwd_rowterm_kernel(const void* o, const v
 // ------------------------------------------------------------------------------------------------
 // shared pieces
 
+// Load of 16 TMEM columns without the wait: the registers are defined only after tmem_wait_ld_pair,
+// which names them as read-write operands so that no use can be scheduled between load and wait.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : FA_R8(0), FA_R8(8)
+      : "r"(taddr)
+      : "memory");
+}
+
+#define FA_RW8(a, i) "+r"(a[i + 0]), "+r"(a[i + 1]), "+r"(a[i + 2]), "+r"(a[i + 3]), "+r"(a[i + 4]), \
+                     "+r"(a[i + 5]), "+r"(a[i + 6]), "+r"(a[i + 7])
+__device__ __forceinline__ void tmem_wait_ld_pair(uint32_t (&a)[16], uint32_t (&b)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : FA_RW8(a, 0), FA_RW8(a, 8), FA_RW8(b, 0), FA_RW8(b, 8)
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               FA_W8(0)
+               : "memory");
+}
+
 __device__ __forceinline__ void smem_desc_pair_k(uint32_t a, uint32_t b, int kk, uint64_t& da, uint64_t& db) {
   // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row; every 4 steps
   // move to the next 64-column panel.  SBO = 8 rows * 128 B.
@@ -335,25 +361,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool masked = (j + 1) * kBT > tile_lim;
       const int lim = row_lim - j * kBT;
+      // the half's 64 key columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
+      uint32_t sb[2][16], db[2][16];
+      tmem_ld16_async(cs, sb[0]);
+      tmem_ld16_async(cd, db[0]);
+      tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int ch = 2 * hh + c2;  // 32-key chunk of the block
-        uint32_t s[32], dp[32], pk[16];
-        tmem_ld32_sync(lane_base + kColS + ch * 32, s);
-        tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
+      for (int c = 0; c < 4; ++c) {
+        const int cur = c & 1;
+        if (c + 1 < 4) {
+          tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
+          tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
+        }
+        uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = ch * 32 + 2 * i;
-          float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, -lse2));
-          float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, -lse2));
+        for (int i = 0; i < 8; ++i) {
+          const int c0 = kHalf * hh + 16 * c + 2 * i;  // key column in the block
+          float p0 = ex2(fmaf(__uint_as_float(sb[cur][2 * i]), sl2, -lse2));
+          float p1 = ex2(fmaf(__uint_as_float(sb[cur][2 * i + 1]), sl2, -lse2));
           if (masked) {
             if (c0 >= lim) p0 = 0.f;
             if (c0 + 1 >= lim) p1 = 0.f;
           }
-          pk[i] = pack2<kFp16>(p0 * (__uint_as_float(dp[2 * i]) - dr), p1 * (__uint_as_float(dp[2 * i + 1]) - dr));
+          pk[i] = pack2<kFp16>(p0 * (__uint_as_float(db[cur][2 * i]) - dr), p1 * (__uint_as_float(db[cur][2 * i + 1]) - dr));
         }
-        // dS over the half's dP, below its unread columns
-        tmem_st16(lane_base + kColDP + kHalf * hh + c2 * 16, pk);
+        tmem_st8(cd + 8 * c, pk);  // dS over the half's dP columns already read
+        if (c + 1 < 4) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -531,33 +565,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       // query already sees the tile's last key
       const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
       const int q_lo = kj - diag - i * kBT;  // columns c < q_lo are masked
+      // the half's 64 query columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
+      uint32_t sb[2][16], db[2][16];
+      tmem_ld16_async(cs, sb[0]);
+      tmem_ld16_async(cd, db[0]);
+      tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int ch = 2 * hh + c2;  // 32-query chunk of the block
-        uint32_t s[32], dp[32], pk[16], dk[16];
-        tmem_ld32_sync(lane_base + kColS + ch * 32, s);
-        tmem_ld32_sync(lane_base + kColDP + ch * 32, dp);
+      for (int c = 0; c < 4; ++c) {
+        const int cur = c & 1;
+        if (c + 1 < 4) {
+          tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
+          tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
+        }
+        uint32_t pk[8], dk[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 l2 = *reinterpret_cast<const float4*>(stat + ch * 32 + 4 * q4);
-          const float4 dr = *reinterpret_cast<const float4*>(stat + kBT + ch * 32 + 4 * q4);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int c0 = kHalf * hh + 16 * c + 4 * q4;  // query column in the block
+          const float4 l2 = *reinterpret_cast<const float4*>(stat + c0);
+          const float4 dr = *reinterpret_cast<const float4*>(stat + kBT + c0);
           const float lv[4] = {l2.x, l2.y, l2.z, l2.w}, dv[4] = {dr.x, dr.y, dr.z, dr.w};
           float pv[4], dsv[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = ch * 32 + 4 * q4 + e;
-            float pe = ex2(fmaf(__uint_as_float(s[4 * q4 + e]), sl2, -lv[e]));
-            if (masked && c < q_lo) pe = 0.f;
+            float pe = ex2(fmaf(__uint_as_float(sb[cur][4 * q4 + e]), sl2, -lv[e]));
+            if (masked && c0 + e < q_lo) pe = 0.f;
             pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(dp[4 * q4 + e]) - dv[e]);
+            dsv[e] = pe * (__uint_as_float(db[cur][4 * q4 + e]) - dv[e]);
           }
           pk[2 * q4] = pack2<kFp16>(pv[0], pv[1]);
           pk[2 * q4 + 1] = pack2<kFp16>(pv[2], pv[3]);
           dk[2 * q4] = pack2<kFp16>(dsv[0], dsv[1]);
           dk[2 * q4 + 1] = pack2<kFp16>(dsv[2], dsv[3]);
         }
-        tmem_st16(lane_base + kColS + kHalf * hh + c2 * 16, pk);   // P^T over the half's S^T
-        tmem_st16(lane_base + kColDP + kHalf * hh + c2 * 16, dk);  // dS^T over the half's dP^T
+        tmem_st8(cs + 8 * c, pk);  // P^T over the half's S^T columns already read
+        tmem_st8(cd + 8 * c, dk);  // dS^T over the half's dP^T columns already read
+        if (c + 1 < 4) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
       }
       tmem_wait_st();
       tc_fence_before();
