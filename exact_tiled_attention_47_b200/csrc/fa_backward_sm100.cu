@@ -44,14 +44,15 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
-constexpr int kStages = 2;
+constexpr int kMaxStages = 3;  // streamed-tile stages: 3 at D = 64, 2 at D = 128 (shared memory)
 constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256;  // S (P over it), dP (dS over it), accumulators
 
 template <int D>
 struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kTileBytes = kBT * D * 2;
-  static constexpr int kUsed = (2 + 2 * kStages) * kTileBytes + 2 * kStages * kBT * 4 + 256 + 1024;
+  static constexpr int kSt = (D == 64) ? 3 : 2;
+  static constexpr int kUsed = (2 + 2 * kSt) * kTileBytes + 2 * kSt * kBT * 4 + 256 + 1024;
   // at least 120 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
   static constexpr int kSmemBytes = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
 };
@@ -71,8 +72,8 @@ struct BwdParams {
 
 struct BwdBars {
   uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
-  uint64_t st_full[kStages], st_empty[kStages];  // streamed tiles (K + V, or Q + dO)
-  uint64_t stat_full[kStages];                   // dK/dV: the streamed block's LSE and Drow in shared memory
+  uint64_t st_full[kMaxStages], st_empty[kMaxStages];  // streamed tiles (K + V, or Q + dO)
+  uint64_t stat_full[kMaxStages];                      // dK/dV: the streamed block's LSE and Drow in shared memory
   uint64_t s_full[2], p_full[2];                 // per half block
   uint64_t o_done, drain;
   uint32_t tmem_base;
@@ -199,7 +200,7 @@ __device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint3
 __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
   if (threadIdx.x == 0) {
     mbar_init(&bars->fixed_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&bars->st_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
       mbar_init(&bars->stat_full[s], 1);
@@ -246,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sDO = smem + C::kTileBytes;
   auto sK = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
-  auto sV = [&](int st) { return smem + (2 + kStages + st) * C::kTileBytes; };
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * kStages) * C::kTileBytes + 2 * kStages * kBT * 4);
+  auto sV = [&](int st) { return smem + (2 + C::kSt + st) * C::kTileBytes; };
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
@@ -287,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        const int st = j % kStages;
-        if (!(ok = mbar_wait(&bars->st_empty[st], ((j / kStages) & 1) ^ 1, abort_flag, p.status))) break;
+        const int st = j % C::kSt;
+        if (!(ok = mbar_wait(&bars->st_empty[st], ((j / C::kSt) & 1) ^ 1, abort_flag, p.status))) break;
         mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         drain_wait(&bars->fixed_full, 0);
-        for (int j = max(0, issued - kStages); j < issued; ++j) drain_wait(&bars->st_full[j % kStages], (j / kStages) & 1);
+        for (int j = max(0, issued - C::kSt); j < issued; ++j) drain_wait(&bars->st_full[j % C::kSt], (j / C::kSt) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(0, 1);
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kStages;
+        const int st = j % C::kSt;
         for (int hh = 0; hh < 2; ++hh) {
           if (!(ok = mbar_wait(&bars->p_full[hh], j & 1, abort_flag, p.status))) break;
           tc_fence_after();
@@ -330,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       j > 0 || hh > 0);
           if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
           if (j + 1 < n) {
-            const int st1 = (j + 1) % kStages;
-            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.status)))
+            const int st1 = (j + 1) % C::kSt;
+            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((j + 1) / C::kSt) & 1, abort_flag, p.status)))
               break;
             tc_fence_after();
             issue_s(st1, hh);
@@ -421,9 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem;
   uint8_t* sV = smem + C::kTileBytes;
   auto sQ = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
-  auto sDO = [&](int st) { return smem + (2 + kStages + st) * C::kTileBytes; };
-  float* sStat = reinterpret_cast<float*>(smem + (2 + 2 * kStages) * C::kTileBytes);  // [stage][lse2 | drow][128]
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * kStages) * C::kTileBytes + 2 * kStages * kBT * 4);
+  auto sDO = [&](int st) { return smem + (2 + C::kSt + st) * C::kTileBytes; };
+  float* sStat = reinterpret_cast<float*>(smem + (2 + 2 * C::kSt) * C::kTileBytes);  // [stage][lse2 | drow][128]
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
@@ -470,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
-      const int i = i_first + jj, st = jj % kStages;
-      if (!(ok = warp_wait(&bars->st_empty[st], ((jj / kStages) & 1) ^ 1, abort_flag, p.status))) break;
+      const int i = i_first + jj, st = jj % C::kSt;
+      if (!(ok = warp_wait(&bars->st_empty[st], ((jj / C::kSt) & 1) ^ 1, abort_flag, p.status))) break;
       if (lane == 0) {  // the tiles first, so their copies overlap the loads of the row statistics
         mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
 #pragma unroll
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok && lane == 0) {
       drain_wait(&bars->fixed_full, 0);
-      for (int jj = max(0, issued - kStages); jj < issued; ++jj) drain_wait(&bars->st_full[jj % kStages], (jj / kStages) & 1);
+      for (int jj = max(0, issued - C::kSt); jj < issued; ++jj) drain_wait(&bars->st_full[jj % C::kSt], (jj / C::kSt) & 1);
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
@@ -524,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(0, 1);
       }
       for (int jj = 0; ok && jj < n; ++jj) {
-        const int st = jj % kStages;
+        const int st = jj % C::kSt;
         for (int hh = 0; hh < 2; ++hh) {
           if (!(ok = mbar_wait(&bars->p_full[hh], jj & 1, abort_flag, p.status))) break;
           tc_fence_after();
@@ -535,8 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       acc);
           if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
           if (jj + 1 < n) {
-            const int st1 = (jj + 1) % kStages;
-            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((jj + 1) / kStages) & 1, abort_flag, p.status)))
+            const int st1 = (jj + 1) % C::kSt;
+            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((jj + 1) / C::kSt) & 1, abort_flag, p.status)))
               break;
             tc_fence_after();
             issue_s(st1, hh);
@@ -555,10 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
-      const int i = i_first + jj, st = jj % kStages;
+      const int i = i_first + jj, st = jj % C::kSt;
       if (!(ok = warp_wait(&bars->s_full[hh], jj & 1, abort_flag, p.status))) break;
       // the stage's LSE/Drow (this stage cannot be refilled before this block's P V products)
-      if (!(ok = warp_wait(&bars->stat_full[st], (jj / kStages) & 1, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(&bars->stat_full[st], (jj / C::kSt) & 1, abort_flag, p.status))) break;
       tc_fence_after();
       const float* stat = sStat + st * 2 * kBT;
       // key kj is visible to query q iff q >= kj - diag (causal); whole block visible iff its first
