@@ -20,7 +20,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 __all__ = [
     "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
-    "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "attention", "decode", "FAError", "LibraryMissing",
+    "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "decode_sharded", "shard_range", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
 ]
 
@@ -289,3 +289,6 @@ def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, works
     if st != FA_OK:
         raise FAError(st, "fa_decode_splitkv" if Hkv == H and seqlens_k is None else "fa_decode_splitkv_gqa")
     return o, lse
+
+
+from .sharded import decode_sharded, shard_range  # noqa: E402  (key-sharded decode over ranks)
