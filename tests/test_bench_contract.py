@@ -1,0 +1,56 @@
+"""The JSON line of bench.py's reference arm (the CPU oracle) carries the keys the benchmark contract
+names (CPU only; the oracle timing itself is replaced by a fixed sample so the test is instant)."""
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_reference_line(monkeypatch, capsys):
+    calls = []
+
+    def fake_sample(cfg, budget, head_iter=None):
+        calls.append(budget)
+        return 2.0e10, 0.5, "fp64 oracle on 1 head (stub)"
+
+    monkeypatch.setattr(bench, "oracle_prefill_sample", fake_sample)
+    monkeypatch.delenv("RANK", raising=False)
+    args = argparse.Namespace(gpus=1, steps=4, warmup=3)
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert len(calls) == 7 and all(b > 0 for b in calls)  # warm-up and timed samples, bounded budgets
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s"
+    assert line["value"] == 2.0e10 / 0.5 / 1e12
+    assert line["config"]["workload"] == bench.HEADLINE
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_other_ranks_do_nothing(monkeypatch, capsys):
+    monkeypatch.setattr(bench, "oracle_prefill_sample", lambda *a, **k: (_ for _ in ()).throw(AssertionError))
+    monkeypatch.setenv("RANK", "1")
+    assert bench.run_reference(argparse.Namespace(gpus=2, steps=2, warmup=3)) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_workload_flops():
+    # 4 B H N^2 D, halved for causal: the headline workload's figure
+    assert bench.prefill_flops(4, 16, 8192, 8192, 64, True) == 549755813888.0
+    assert bench.prefill_flops(1, 1, 128, 256, 64, False) == 4 * 128 * 256 * 64
+
+
+def test_prefix_flops_counts_visible_pairs():
+    # 4 D FLOPs per visible (query, key) pair; the prefix-LM pair count by brute force
+    N, D = 37, 64
+    for p in (0, 1, 10, 36, 37):
+        pairs = sum(1 for i in range(N) for j in range(N) if j < p or j <= i)
+        assert bench.prefix_flops(2, 3, N, D, p) == 2 * 3 * 4 * D * pairs
