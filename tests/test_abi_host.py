@@ -238,3 +238,24 @@ def test_no_device_is_reported(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(fa.LibraryMissing):
         fa._lib.load(str(tmp_path / "nope.so"))
+
+
+def test_plain_c_program(lib, tmp_path):
+    """The boundary is usable from C99 alone: tests/c_abi_check.c compiled with gcc against
+    include/fa.h and linked to the built library (no CUDA headers, no C++, no torch)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(fa.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    src = os.path.join(ROOT, "tests", "c_abi_check.c")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                        "-L", libdir, "-lfa_sm100", "-Wl,-rpath," + libdir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    import torch
+    args = [] if torch.cuda.is_available() else ["nodevice"]
+    r = subprocess.run([exe] + args, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "c_abi_check: ok" in r.stdout
