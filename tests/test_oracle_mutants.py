@@ -1,0 +1,83 @@
+"""Mutation check of the oracle pins (CPU only).
+
+Each case plants one plausible slip in a private copy of the oracle (a dropped scale, an off-by-one or
+mis-aligned mask, a wrong log base, a missing normalisation, a sign flip, a broken merge or gradient
+term) and runs the oracle pins against that copy: every mutant must make them fail, while the
+unmodified copy must pass.  The repository's own files are never edited.
+"""
+import os
+import shutil
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# (file under oracle/, text to replace, replacement)
+MUTANTS = {
+    "drop_scale": ("attention.py", "s = scale * (q @ k.T)", "s = (q @ k.T)"),
+    "causal_off_by_one": ("attention.py", "vis &= (j <= i + (nk - nq)) | (j < prefix)",
+                          "vis &= (j < i + (nk - nq)) | (j < prefix)"),
+    "causal_top_left": ("attention.py", "vis &= (j <= i + (nk - nq)) | (j < prefix)",
+                        "vis &= (j <= i) | (j < prefix)"),
+    "prefix_off_by_one": ("attention.py", "vis &= (j <= i + (nk - nq)) | (j < prefix)",
+                          "vis &= (j <= i + (nk - nq)) | (j <= prefix)"),
+    "key_length_off_by_one": ("attention.py", "vis &= j < k_valid", "vis &= j <= k_valid"),
+    "lse_log2": ("attention.py", "lse[live] = m + np.log(l)", "lse[live] = m + np.log2(l)"),
+    "lse_without_max": ("attention.py", "lse[live] = m + np.log(l)", "lse[live] = np.log(l)"),
+    "no_normalisation": ("attention.py", "o[live] = (p @ v) / l[:, None]", "o[live] = (p @ v)"),
+    "exp_sign": ("attention.py", "p = np.exp(sl - m[:, None])", "p = np.exp(m[:, None] - sl)"),
+    "shard_offset_sign": ("attention.py", "min(max(int(L) - key_offset, 0), nk)",
+                          "min(max(int(L) + key_offset, 0), nk)"),
+    "tiled_no_rescale": ("online.py", "acc = alpha[:, None] * acc + p @ vj", "acc = acc + p @ vj"),
+    "merge_drops_weight": ("online.py", "return m, np.concatenate([e1 * f1, e2 * f2]), e1 * l1 + e2 * l2",
+                           "return m, np.concatenate([f1, e2 * f2]), l1 + e2 * l2"),
+    "combine_old_weight": ("online.py", "acc = e_old * acc + e_s * o_s", "acc = acc + e_s * o_s"),
+    "bwd_drop_row_term": ("backward.py", "ds = p * (dp - drow[:, None])", "ds = p * dp"),
+    "bwd_dq_no_scale": ("backward.py", "dq = scale * (ds @ k)", "dq = ds @ k"),
+    "bwd_dk_transposed": ("backward.py", "dk = scale * (ds.T @ q)", "dk = scale * (ds @ q)[: q.shape[0]]"),
+}
+
+
+def _tree(dst):
+    """A private copy of what the pins need: the oracle, the input generator and the pins."""
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"),
+                    ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "seeded_inputs.py"), dst)
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), dst)
+    os.makedirs(os.path.join(dst, "tests"))
+    for f in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests", f))
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
+
+
+def _run_pins(dst):
+    env = dict(os.environ, PYTHONPATH=dst, PYTHONDONTWRITEBYTECODE="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "tests/test_oracle_pins.py"], cwd=dst,
+                       env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode, (r.stdout.strip().splitlines() or [""])[-1]
+
+
+def _case(base, name):
+    dst = os.path.join(base, name)
+    _tree(dst)
+    if name != "unmodified":
+        fname, old, new = MUTANTS[name]
+        path = os.path.join(dst, "oracle", fname)
+        src = open(path).read()
+        assert src.count(old) == 1, f"{name}: anchor not found once in oracle/{fname}"
+        open(path, "w").write(src.replace(old, new))
+    return name, _run_pins(dst)
+
+
+@pytest.mark.slow
+def test_every_mutant_fails_the_pins(tmp_path):
+    names = ["unmodified"] + list(MUTANTS)
+    with ThreadPoolExecutor(min(8, os.cpu_count() or 1)) as ex:
+        results = dict(ex.map(lambda n: _case(str(tmp_path), n), names))
+    rc, last = results.pop("unmodified")
+    assert rc == 0, f"the unmodified copy must pass: {last}"
+    survivors = {n: last for n, (rc, last) in results.items() if rc == 0}
+    assert not survivors, f"mutants not caught by the pins: {survivors}"
