@@ -263,6 +263,31 @@ def sharded_leg(args, kc, vc, dev, rank, world, dist, pk, pk_kind, fa, torch, st
             "gpu_launches": 3 * steps}
 
 
+def add_token_rates(line, world):
+    """Tokens per second beside the FLOP and byte rates: prefill B*N query tokens per step, decode one
+    token per sequence per step, all ranks together (max-over-ranks step time).  Never raises: a
+    missing figure just leaves the key out."""
+    def rate(tokens, ms):
+        return tokens / (ms * 1e-3) if tokens and ms else None
+
+    try:
+        cfg = line.get("config") or {}
+        if line.get("ms_per_step"):
+            line["tokens_per_s"] = rate(cfg["B"] * cfg["N"] * world, line["ms_per_step"])
+        dec = line.get("decode") or {}
+        if dec.get("ms_per_step"):
+            dec["tokens_per_s"] = rate(dec["config"]["B"] * world, dec["ms_per_step"])
+        for key in ("gqa", "sharded"):
+            sub = dec.get(key) or {}
+            if sub.get("ms_per_step"):
+                # the sharded cache is one problem split over the ranks: its B sequences per step
+                n = sub["config"]["B"] * (world if key == "gqa" else 1)
+                sub["tokens_per_s"] = rate(n, sub["ms_per_step"])
+    except (KeyError, TypeError, ZeroDivisionError):
+        pass
+    return line
+
+
 def timed_run(run, steps, stream, dist=None):
     """Time run(steps), which may use other streams but joins them into `stream` before it returns."""
     import torch
@@ -698,6 +723,7 @@ def main():
         "gpu_launches": args.steps if run_prefill else 0,
         "decode": dec, "prefix": prefix, "backward": bwd, "cpu_baseline": cpu,
     }
+    add_token_rates(line, world)
     print(json.dumps(line), flush=True)
     return 0
 
