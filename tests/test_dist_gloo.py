@@ -82,7 +82,7 @@ def _shard_worker(rank, world, port, out):
         import seeded_inputs as si
         from exact_tiled_attention_47_b200.sharded import gather_parts, part_floats, shard_range
         B, Hq, Hkv, Nk, D, scale = 3, 4, 2, 37, 64, 0.125
-        lens = [37, 18, 0]  # the second ends inside shard 0 of 2 (keys 0..18), the third is empty
+        lens = [37, 18, 0]  # the second ends inside the first shard (2 ranks) or the second (3), the third is empty
         qb, kb, vb = si.decode_gqa_inputs(41, B, Nk, Hq, Hkv, D, "bf16")
         q, k, v = (si.bits_to_float(t, "bf16") for t in (qb, kb, vb))
         off, n = shard_range(Nk, world, rank)
@@ -112,8 +112,8 @@ def _shard_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_sharded_decode_exchange_gloo():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_decode_exchange_gloo(world):
     port = _free_port()
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
@@ -124,7 +124,11 @@ def test_sharded_decode_exchange_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert [r[1] for r in res] == [(0, 19), (19, 18)]   # contiguous shards covering 37 keys
+    bounds = [r[1] for r in res]                      # contiguous shards covering the 37 keys
+    assert bounds[0][0] == 0 and bounds[-1][0] + bounds[-1][1] == 37
+    assert all(a[0] + a[1] == b[0] for a, b in zip(bounds, bounds[1:]))
+    if world == 2:
+        assert bounds == [(0, 19), (19, 18)]
     for _, _, err_o, err_l, own_block_in_place in res:
         assert own_block_in_place                       # block r of the gather is rank r's
         assert err_o < 1e-6 and err_l < 1e-6            # fp32 packing is the only rounding
