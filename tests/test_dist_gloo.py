@@ -147,3 +147,80 @@ def test_shard_ranges_cover_the_cache():
         shard_range(3, 4, 0)
     with pytest.raises(ValueError):
         shard_range(10, 2, 2)
+
+
+def _decode_sharded_worker(rank, world, port, out):
+    """One rank calling the public helper decode_sharded on CPU tensors.  Its two library calls are
+    replaced by stand-ins computed with the oracle that honour the documented block layout (the
+    shard's fp32 O [B,H,D] then LSE [B,H], padded to 16 bytes; blocks in rank order), so what is
+    tested is the helper itself: part sizing, layout, the all-gather and the merge call."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import seeded_inputs as si
+        import exact_tiled_attention_47_b200 as fa
+        from exact_tiled_attention_47_b200.sharded import decode_sharded, shard_range
+        B, Hq, Hkv, Nk, D, scale = 2, 4, 2, 50, 64, 0.2
+        lens = [50, 23]
+        qb, kb, vb = si.decode_gqa_inputs(43, B, Nk, Hq, Hkv, D, "bf16")
+        q, k, v = (si.bits_to_float(t, "bf16") for t in (qb, kb, vb))
+        calls = {}
+
+        def fake_shard(q_, k_, v_, part, B_, Hq_, Hkv_, Nk_shard, key_offset, Nk_total, D_, scale_, S_, sl, ws,
+                       workspace_bytes=None, stream=None, in_dtype=None):
+            calls["shard"] = (Nk_shard, key_offset, Nk_total)
+            o_r, l_r = oracle.attention_decode_shard(q_.double().numpy(), k_.double().numpy(), v_.double().numpy(),
+                                                     scale_, key_offset, None if sl is None else sl.tolist())
+            part[:B_ * Hq_ * D_] = torch.from_numpy(o_r.reshape(-1)).float()
+            part[B_ * Hq_ * D_:B_ * Hq_ * (D_ + 1)] = torch.from_numpy(l_r.reshape(-1)).float()
+            return 0
+
+        def fake_merge(parts, R, B_, H_, D_, o, lse, stream=None, o_dtype=None):
+            calls["merge"] = (R, parts.numel())
+            nf = parts.numel() // R
+            blocks = parts.view(R, nf).double().numpy()
+            for row in range(B_ * H_):
+                ob, lb = oracle.combine_partials([blk[row * D_:(row + 1) * D_] for blk in blocks],
+                                                 [blk[B_ * H_ * D_ + row] for blk in blocks])
+                o.view(B_ * H_, D_)[row] = torch.from_numpy(ob).to(o.dtype)
+                lse.view(-1)[row] = float(lb)
+            return 0
+
+        fa.fa_decode_splitkv_shard = fake_shard
+        fa.fa_decode_merge = fake_merge
+        off, n = shard_range(Nk, world, rank)
+        qt = torch.from_numpy(q).float()
+        kt = torch.from_numpy(np.ascontiguousarray(k[:, off:off + n])).float()
+        vt = torch.from_numpy(np.ascontiguousarray(v[:, off:off + n])).float()
+        o, lse = decode_sharded(qt, kt, vt, off, Nk, scale=scale, num_splits=4,
+                                seqlens_k=torch.tensor(lens, dtype=torch.int32), out_dtype=torch.float32)
+        o_ref, lse_ref = oracle.attention_decode_gqa(q, k, v, scale, lens)
+        out.put((rank, calls["shard"], calls["merge"], float(np.abs(o.numpy() - o_ref).max()),
+                 float(np.abs(lse.numpy() - lse_ref).max())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_decode_sharded_helper_gloo():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_decode_sharded_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(out.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    from exact_tiled_attention_47_b200.sharded import part_floats
+    for rank, shard, merge, err_o, err_l in res:
+        assert shard == ((25, 25 * rank, 50))                      # this rank's keys of the 50-key cache
+        assert merge == (2, 2 * part_floats(2, 4, 64))             # both ranks' blocks, one merge
+        assert err_o < 1e-6 and err_l < 1e-6                       # fp32 blocks are the only rounding
