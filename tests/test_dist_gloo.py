@@ -208,6 +208,8 @@ def _decode_sharded_worker(rank, world, port, out):
 
 
 def test_decode_sharded_helper_gloo():
+    from exact_tiled_attention_47_b200 import build
+    build.build()  # the helper sizes its buffers through the library's host functions
     world = 2
     port = _free_port()
     ctx = mp.get_context("spawn")
