@@ -13,7 +13,8 @@ Modules:
                 inside, running max m and running sum l), and the pairwise merge of softmax
                 statistics of key groups, including the split-KV partial/combine form.
   brute      -- scalar pure-Python (math.fsum) evaluation for tiny inputs.
-  backward   -- dQ, dK, dV: the derivative of the forward definition for an upstream gradient dO.
+  backward   -- dQ, dK, dV: the derivative of the forward definition for an upstream gradient dO
+                (whole head, dense, packed varlen, and at sampled rows of long heads).
 """
 from .attention import (attention_head, attention_dense, attention_varlen, attention_rows,
                         attention_decode, attention_decode_gqa, attention_decode_shard,
@@ -21,12 +22,14 @@ from .attention import (attention_head, attention_dense, attention_varlen, atten
 from .online import (tiled_online_attention, group_stats, merge_groups, softmax_by_groups,
                      split_kv_partials, combine_partials)
 from .brute import brute_attention_head
-from .backward import attention_head_backward, attention_dense_backward, backward_row_terms
+from .backward import (attention_head_backward, attention_dense_backward, attention_varlen_backward,
+                       attention_rows_backward)
 
 __all__ = [
     "attention_head", "attention_dense", "attention_varlen", "attention_rows", "attention_decode",
     "attention_decode_gqa", "attention_decode_shard",
     "padded_key_mask_attention", "tiled_online_attention", "group_stats", "merge_groups",
     "softmax_by_groups", "split_kv_partials", "combine_partials", "brute_attention_head",
-    "attention_head_backward", "attention_dense_backward", "backward_row_terms",
+    "attention_head_backward", "attention_dense_backward", "attention_varlen_backward",
+    "attention_rows_backward",
 ]

@@ -29,14 +29,16 @@ from __future__ import annotations
 import numpy as np
 
 
-def _visible_mask(nq: int, nk: int, causal: bool, k_valid: int | None, prefix: int = 0) -> np.ndarray:
-    """Boolean [nq, nk]: True where query i may attend to key j."""
+def _visible_mask(nq: int, nk: int, causal: bool, k_valid: int | None, prefix: int = 0,
+                  row_lo: int = 0, row_hi: int | None = None) -> np.ndarray:
+    """Boolean [rows, nk]: True where query i (rows row_lo..row_hi-1, default all) may attend to key j."""
+    row_hi = nq if row_hi is None else row_hi
     j = np.arange(nk)[None, :]
-    vis = np.ones((nq, nk), dtype=bool)
+    vis = np.ones((row_hi - row_lo, nk), dtype=bool)
     if k_valid is not None:
         vis &= j < k_valid
     if causal:
-        i = np.arange(nq)[:, None]
+        i = np.arange(row_lo, row_hi)[:, None]
         vis &= (j <= i + (nk - nq)) | (j < prefix)
     return vis
 

@@ -91,38 +91,6 @@ def test_backward_deterministic():
         assert torch.equal(a, b)
 
 
-def _head_rows(qh, kh, vh, doh, scale, rows, cols):
-    """Oracle gradients of one causal head at sampled query rows (dQ) and key rows (dK, dV), fp64."""
-    n = qh.shape[0]
-    # LSE of every row, 512 rows at a time (keys j <= i visible)
-    lse = np.empty(n)
-    for a in range(0, n, 512):
-        s = scale * (qh[a:a + 512] @ kh.T)
-        i = np.arange(a, min(n, a + 512))[:, None]
-        s = np.where(np.arange(n)[None, :] <= i, s, -np.inf)
-        m = s.max(axis=1)
-        lse[a:a + 512] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
-    # O and the row term for every row (dQ and dK need Drow_i of every query)
-    drow = np.empty(n)
-    for a in range(0, n, 512):
-        s = scale * (qh[a:a + 512] @ kh.T)
-        i = np.arange(a, min(n, a + 512))[:, None]
-        p = np.where(np.arange(n)[None, :] <= i, np.exp(s - lse[a:a + 512, None]), 0.0)
-        drow[a:a + 512] = ((p @ vh) * doh[a:a + 512]).sum(axis=1)
-    dq = []
-    for i in rows:
-        p = np.exp(scale * (kh[:i + 1] @ qh[i]) - lse[i])
-        ds = p * (vh[:i + 1] @ doh[i] - drow[i])
-        dq.append(scale * (ds @ kh[:i + 1]))
-    dk, dv = [], []
-    for j in cols:
-        p = np.exp(scale * (qh[j:] @ kh[j]) - lse[j:])  # queries i >= j see key j
-        ds = p * (doh[j:] @ vh[j] - drow[j:])
-        dk.append(scale * (ds @ qh[j:]))
-        dv.append(p @ doh[j:])
-    return np.array(dq), np.array(dk), np.array(dv)
-
-
 def test_backward_full_size_sampled():
     import exact_tiled_attention_47_b200 as fa
     c = si.CONFIGS["prefill_d64"]
@@ -143,7 +111,7 @@ def test_backward_full_size_sampled():
     rows = np.unique(np.concatenate([[0, 1, 127, 128, 4095, N - 1], rng.integers(0, N, 10)]))
     for b, h in [(0, 0), (B - 1, H - 1)]:
         f = lambda x: to_f64(x[b, :, h], dt)
-        rq, rk, rv = _head_rows(f(q), f(k), f(v), f(do), scale, rows, rows)
+        rq, rk, rv = oracle.attention_rows_backward(f(q), f(k), f(v), f(do), scale, rows, rows, causal=True)
         for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             gn = g[b, :, h].cpu().numpy().astype(np.float64)[rows]
             m = max(np.abs(r).max(), 1e-6)

@@ -38,6 +38,15 @@ MUTANTS = {
     "bwd_drop_row_term": ("backward.py", "ds = p * (dp - drow[:, None])", "ds = p * dp"),
     "bwd_dq_no_scale": ("backward.py", "dq = scale * (ds @ k)", "dq = ds @ k"),
     "bwd_dk_transposed": ("backward.py", "dk = scale * (ds.T @ q)", "dk = scale * (ds @ q)[: q.shape[0]]"),
+    "bwd_prefix_ignored": ("backward.py", "q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale, causal, prefix)",
+                           "q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale, causal, 0)"),
+    "bwd_varlen_prefix_ignored": ("backward.py", "do[s0:s1, h], scale, causal, prefix)",
+                                  "do[s0:s1, h], scale, causal, 0)"),
+    "bwd_rows_drop_row_term": ("backward.py", "dsc = pc * (do[a:e] @ v[cols].T - drow[:, None])",
+                               "dsc = pc * (do[a:e] @ v[cols].T)"),
+    "bwd_rows_chunk_offset": ("attention.py", "i = np.arange(row_lo, row_hi)[:, None]",
+                              "i = np.arange(0, row_hi - row_lo)[:, None]"),
+    "bwd_rows_dv_uses_ds": ("backward.py", "dv += pc.T @ do[a:e]", "dv += dsc.T @ do[a:e]"),
 }
 
 

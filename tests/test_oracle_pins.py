@@ -26,8 +26,10 @@ wrong LSE base, a bad group merge) fails at least one of them:
     the split-KV combine with empty splits;
   * decode over key shards of a cache: the Q = 0 closed form with the shard's own visible-key
     count, and the merge of all shards' results equal to decode over the whole cache;
-  * the backward (dQ, dK, dV): central finite differences of the forward oracle, the Q = 0 closed
-    forms, invariance of dQ and dV under a common key shift, and zero total dK.
+  * the backward (dQ, dK, dV): central finite differences of the forward oracle (causal, unmasked,
+    prefix-LM, and the packed varlen form), the Q = 0 closed forms, invariance of dQ and dV under a
+    common key shift, and zero total dK; the row-sampled backward for long heads equals the
+    whole-head backward at every row and column.
 """
 import json
 import math
@@ -493,30 +495,95 @@ def test_shard_decode_zero_query_closed_form():
 # backward: the derivative of the forward definition
 
 
-def _loss(q, k, v, do, scale, causal):
-    o, _ = oracle.attention_head(q, k, v, scale, causal)
+def _loss(q, k, v, do, scale, causal, prefix=0):
+    o, _ = oracle.attention_head(q, k, v, scale, causal, prefix=prefix)
     return float((o * do).sum())
 
 
-@pytest.mark.parametrize("nq,nk,causal", [(6, 6, False), (7, 7, True), (5, 9, True), (9, 5, True), (4, 11, False)])
-def test_backward_matches_finite_differences(nq, nk, causal):
-    # central differences of the (pinned) forward oracle: error O(h^2) ~ 1e-10 for h = 1e-5
-    d, dv_, scale, h = 5, 4, 0.4, 1e-5
-    rng = np.random.default_rng(nq * 31 + nk)
-    q, k, v = rng.standard_normal((nq, d)), rng.standard_normal((nk, d)), rng.standard_normal((nk, dv_))
-    do = rng.standard_normal((nq, dv_))
-    dq, dk, dv = oracle.attention_head_backward(q, k, v, do, scale, causal)
-    for x, g in ((q, dq), (k, dk), (v, dv)):
+def _central_differences(loss, tensors, h=1e-5):
+    """d loss / d x for every element of every tensor (edited in place and restored)."""
+    out = []
+    for x in tensors:
         num = np.zeros_like(x)
         for idx in np.ndindex(x.shape):
             keep = x[idx]
             x[idx] = keep + h
-            lp = _loss(q, k, v, do, scale, causal)
+            lp = loss()
             x[idx] = keep - h
-            lm = _loss(q, k, v, do, scale, causal)
+            lm = loss()
             x[idx] = keep
             num[idx] = (lp - lm) / (2 * h)
+        out.append(num)
+    return out
+
+
+@pytest.mark.parametrize("nq,nk,causal,prefix", [(6, 6, False, 0), (7, 7, True, 0), (5, 9, True, 0), (9, 5, True, 0),
+                                                  (4, 11, False, 0), (7, 7, True, 3), (5, 9, True, 6),
+                                                  (9, 5, True, 2)])
+def test_backward_matches_finite_differences(nq, nk, causal, prefix):
+    # central differences of the (pinned) forward oracle: error O(h^2) ~ 1e-10 for h = 1e-5
+    d, dv_, scale = 5, 4, 0.4
+    rng = np.random.default_rng(nq * 31 + nk + 101 * prefix)
+    q, k, v = rng.standard_normal((nq, d)), rng.standard_normal((nk, d)), rng.standard_normal((nk, dv_))
+    do = rng.standard_normal((nq, dv_))
+    grads = oracle.attention_head_backward(q, k, v, do, scale, causal, prefix)
+    nums = _central_differences(lambda: _loss(q, k, v, do, scale, causal, prefix), (q, k, v))
+    for g, num in zip(grads, nums):
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal,prefix", [(False, 0), (True, 0), (True, 4)])
+def test_dense_backward_matches_finite_differences(causal, prefix):
+    # the [B, N, H, D] layout: every (batch, head) differentiated with its own mask (prefix 4 widens
+    # rows 0-2, which see keys 0..i+1 under the causal mask alone)
+    B, nq, nk, H, d, scale = 2, 5, 6, 2, 3, 0.6
+    rng = np.random.default_rng(23 + prefix + 7 * causal)
+    q, do = rng.standard_normal((B, nq, H, d)), rng.standard_normal((B, nq, H, d))
+    k, v = rng.standard_normal((B, nk, H, d)), rng.standard_normal((B, nk, H, d))
+
+    def loss():
+        o, _ = oracle.attention_dense(q, k, v, scale, causal, prefix)
+        return float((o * do).sum())
+
+    grads = oracle.attention_dense_backward(q, k, v, do, scale, causal, prefix)
+    nums = _central_differences(loss, (q, k, v))
+    for g, num in zip(grads, nums):
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal,prefix", [(False, 0), (True, 0), (True, 2)])
+def test_varlen_backward_matches_finite_differences(causal, prefix):
+    # packed sequences (one empty); the loss is taken over the packed forward oracle's output
+    lengths, H, d, scale = [3, 0, 5, 1, 4], 2, 3, 0.7
+    cu = si.cu_seqlens_of(lengths)
+    total = int(cu[-1])
+    rng = np.random.default_rng(17 + prefix + 5 * causal)
+    q, k, v, do = (rng.standard_normal((total, H, d)) for _ in range(4))
+
+    def loss():
+        o, _ = oracle.attention_varlen(q, k, v, cu, scale, causal, prefix)
+        return float((o * do).sum())
+
+    grads = oracle.attention_varlen_backward(q, k, v, do, cu, scale, causal, prefix)
+    nums = _central_differences(loss, (q, k, v))
+    for g, num in zip(grads, nums):
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("nq,nk,causal,prefix,chunk", [(40, 40, False, 0, 7), (45, 45, True, 0, 8),
+                                                        (30, 52, True, 0, 16), (52, 30, True, 0, 5),
+                                                        (41, 41, True, 9, 6), (33, 50, False, 0, 64)])
+def test_row_sampled_backward_matches_whole_head(nq, nk, causal, prefix, chunk):
+    # every row and column sampled, query rows visited in blocks smaller than the head
+    d, scale = 6, 0.35
+    rng = np.random.default_rng(nq + 3 * nk + prefix)
+    q, k, v, do = (rng.standard_normal(s) for s in ((nq, d), (nk, d), (nk, d), (nq, d)))
+    dq, dk, dv = oracle.attention_head_backward(q, k, v, do, scale, causal, prefix)
+    rows, cols = np.arange(nq)[::-1], np.arange(nk)[::-1]  # any order, returned in the order asked
+    rq, rk, rv = oracle.attention_rows_backward(q, k, v, do, scale, rows, cols, causal, prefix, chunk=chunk)
+    np.testing.assert_allclose(rq, dq[rows], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(rk, dk[cols], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(rv, dv[cols], rtol=1e-11, atol=1e-13)
 
 
 def test_backward_closed_forms():
