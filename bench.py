@@ -99,7 +99,7 @@ def causal_rows_flops(rows_lo, rows_hi, N, D):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons of one GPU with NVML every ~20 ms (read-only)."""
+    """Samples SM clock and throttle reasons of one GPU with NVML every ~2 ms (read-only)."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
@@ -107,8 +107,9 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index):
+    def __init__(self, index, period_s=0.002):
         self.index = index
+        self.period_s = period_s
         self.samples = []
         self.reasons = set()
         self._stop = threading.Event()
@@ -142,7 +143,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(self.period_s)
 
     def __exit__(self, *exc):
         self._stop.set()
@@ -392,6 +393,78 @@ def run_reference(args):
 # our arm
 
 
+def varlen_flops(lengths, H, D, causal=False):
+    """Sum over packed sequences of 4 * H * L^2 * D (halved for causal)."""
+    f = sum(4.0 * H * int(L) * int(L) * D for L in lengths)
+    return f / 2 if causal else f
+
+
+def other_prefill_leg(args, name, dev, rank, world, dist, pk, pk_kind, fa, torch):
+    """One more prefill workload (the other head dim, or the packed varlen encoder) timed the same way
+    as the headline: CUDA events over the timed steps, inputs larger than L2.  Returns a sub-line."""
+    cfg = si.CONFIGS[name]
+    stream = torch.cuda.current_stream(dev)
+    seed = rank_seed(cfg["seed"], rank)
+    dt, H, D, scale = cfg["dtype"], cfg["H"], cfg["D"], cfg["scale"]
+    causal = bool(cfg.get("causal", False))
+    if name == "varlen":
+        lengths = si.varlen_lengths(cfg["seed"], cfg["nseq"], cfg["len_lo"], cfg["len_hi"])
+        q, k, v, cu = si.varlen_qkv(seed, lengths, H, D, dt)
+        total = int(cu[-1])
+        B, Nq = len(lengths), total
+        cud = torch.from_numpy(cu).to(dev)
+        flops = varlen_flops(lengths, H, D, causal)
+        tokens = total
+        lse = torch.empty((H, total), dtype=torch.float32, device=dev)
+        conf = {"workload": name, "sequences": B, "total_tokens": total,
+                "lengths": f"U{{{cfg['len_lo']}..{cfg['len_hi']}}} seeded", "H": H, "D": D, "causal": causal,
+                "input_dtype": dt, "output_dtype": dt, "scale": scale}
+    else:
+        B, Nq = cfg["B"], cfg["Nq"]
+        q, k, v = si.dense_qkv(seed, B, Nq, Nq, H, D, dt)
+        cud = None
+        flops = prefill_flops(B, H, Nq, Nq, D, causal)
+        tokens = B * Nq
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+        conf = {"workload": name, "B": B, "H": H, "N": Nq, "D": D, "causal": causal, "input_dtype": dt,
+                "output_dtype": dt, "scale": scale}
+    qd, kd, vd = (to_dev(t, dt, dev) for t in (q, k, v))
+    del q, k, v
+    od = torch.empty_like(qd)
+    conf["l2"] = f"inputs {3 * qd.numel() * 2 / 2**20:.0f} MiB > 126 MB L2 (no flush needed)"
+
+    def step():
+        st = fa.fa_fwd(qd, kd, vd, od, lse, B, H, Nq, Nq, D, scale, causal, cud, stream)
+        if st:
+            raise fa.FAError(st, "fa_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(10, min(args.steps, 50))
+    with ClockSampler(dev.index) as clk:
+        ms = timed(step, steps, stream, dist)
+    if fa.fa_device_status(clear=True) != 0:
+        raise RuntimeError(f"device status set during the timed {name} run")
+    ms_step = ms / steps
+    tf = flops / (ms_step * 1e-3) / 1e12
+    dtn = "fp16" if dt == "fp16" else "bf16"
+    out = {"metric": "attention fwd TFLOPS", "value": whole_job_rate(flops, ms_step, world) / 1e12,
+           "unit": "TFLOP/s", "ms_per_step": ms_step, "steps": steps,
+           "tokens_per_s": tokens * world / (ms_step * 1e-3), "config": conf,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": tf / pk["bf16_tflops"], "traffic": measured_traffic(name),
+                        "traffic_unit": "bytes per launch (ncu dram read+write)",
+                        "kernel": f"fa_fwd_kernel<{D},{dtn},out {dtn}>",
+                        "peak_kind": f"{pk_kind} bf16 burst (fp16 has the same dense rate)",
+                        "frac_of_sustained": tf / pk["bf16_tflops_sustained"],
+                        "algorithmic_flops_per_launch": flops},
+           "clocks": clk.summary(), "gpu_launches": steps}
+    del qd, kd, vd, od, lse
+    torch.cuda.empty_cache()
+    return out
+
+
 def prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind, fa, torch):
     """Time the headline prefill workload; returns (value, ms_step, roofline, e2e, clocks, prefix)."""
     B, N, H, D, dt = cfg["B"], cfg["Nq"], cfg["H"], cfg["D"], cfg["dtype"]
@@ -561,9 +634,12 @@ def main():
     ap.add_argument("--no-prefix", action="store_true", help="skip the prefix-mask timing of the prefill inputs")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing of the prefill inputs")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the timing of the other prefill workloads (the other head dim, varlen)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="profiling runs: time only one of the two paths")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "varlen", "other"], default="all",
+                    help="profiling runs: time only the headline prefill, the decode legs, the varlen leg, "
+                         "or the other head dim's prefill leg")
     ap.add_argument("--workload", choices=["prefill_d64", "prefill_d128"], default=HEADLINE,
                     help="prefill workload of the headline leg (default: the D=64 configuration)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -604,6 +680,16 @@ def main():
     if run_prefill:
         value, ms_step, roof, e2e, clk, prefix, bwd = prefill_leg(args, cfg, dev, rank, world, dist, pk, pk_kind,
                                                                   fa, torch)
+
+    # ---------------- the other prefill workloads ----------------
+    others = {}
+    if not args.no_others:
+        other = "prefill_d128" if args.workload == "prefill_d64" else "prefill_d64"
+        if args.only in ("all", "other"):
+            others["p128" if other == "prefill_d128" else "p64"] = other_prefill_leg(
+                args, other, dev, rank, world, dist, pk, pk_kind, fa, torch)
+        if args.only in ("all", "varlen"):
+            others["varlen"] = other_prefill_leg(args, "varlen", dev, rank, world, dist, pk, pk_kind, fa, torch)
 
     # ---------------- decode (secondary metric) ----------------
     dec = None
@@ -723,6 +809,7 @@ def main():
         "gpu_launches": args.steps if run_prefill else 0,
         "decode": dec, "prefix": prefix, "backward": bwd, "cpu_baseline": cpu,
     }
+    line.update(others)
     add_token_rates(line, world)
     print(json.dumps(line), flush=True)
     return 0

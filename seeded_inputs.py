@@ -175,6 +175,32 @@ def decode_gqa_inputs(seed: int, B: int, Nk: int, Hq: int, Hkv: int, D: int, dty
     return q, k, v
 
 
+def key_ramp(q: np.ndarray, k: np.ndarray, dtype: str, q_value: float, top: float, key_axis: int,
+             cu_seqlens=None):
+    """Copies of Q and K (uint16 bits) with channel 0 replaced to give scores that rise along the keys.
+
+    Channel 0 of every query becomes ``q_value`` and channel 0 of key j becomes ``top * j / (n - 1)``,
+    j counted along ``key_axis`` of K (from the start of each packed sequence when ``cu_seqlens`` is
+    given, the key axis being axis 0 then).  Only the inputs' structure changes: the last channel
+    index is the head dimension, all other channels keep their random values.
+    """
+    q2, k2 = q.copy(), k.copy()
+    q2[..., 0] = round_to_bits(np.full(q2.shape[:-1], q_value, dtype=np.float32), dtype)
+    kc = np.moveaxis(k2[..., 0], key_axis, 0)  # view: keys first
+    if cu_seqlens is None:
+        spans = [(0, kc.shape[0])]
+    else:
+        spans = [(int(a), int(b)) for a, b in zip(cu_seqlens[:-1], cu_seqlens[1:])]
+    for a, b in spans:
+        n = b - a
+        if n <= 0:
+            continue
+        ramp = (np.arange(n, dtype=np.float32) * np.float32(top / max(n - 1, 1))).astype(np.float32)
+        vals = np.broadcast_to(ramp.reshape((n,) + (1,) * (kc.ndim - 1)), (n,) + kc.shape[1:])
+        kc[a:b] = round_to_bits(np.ascontiguousarray(vals), dtype)
+    return q2, k2
+
+
 def config_inputs(name: str, **overrides):
     """Inputs of one named workload (optionally with smaller sizes for the oracle)."""
     c = dict(CONFIGS[name])

@@ -57,3 +57,31 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, out_dtype="fp32", what=""):
                max_dlse=float(dl.max(initial=0.0)), bad_o=bad_o, bad_lse=bad_l)
     assert bad_o == 0 and bad_l == 0, f"{what}: {rep}"
     return rep
+
+
+GUARD_BYTES = 4096  # sentinel bytes before and after a guarded buffer (keeps 16-byte alignment)
+GUARD_FILL = 0xA5
+
+
+class Guarded:
+    """A device tensor with sentinel-filled guard bands on both sides (canaries for stray writes).
+
+    ``t`` is the tensor the kernel gets; ``intact()`` checks that not one byte of either band (nor
+    of the padding up to the next 256 bytes) changed.  The tensor itself starts filled with the
+    sentinel too, so any element a kernel forgets to write is visible as well.
+    """
+
+    def __init__(self, shape, dtype, device="cuda"):
+        import torch
+        shape = tuple(int(x) for x in shape)
+        elem = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = int(np.prod(shape, dtype=np.int64)) * elem
+        padded = (self.nbytes + 255) // 256 * 256
+        self.raw = torch.full((2 * GUARD_BYTES + padded,), GUARD_FILL, dtype=torch.uint8, device=device)
+        self.t = self.raw[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(shape)
+
+    def intact(self) -> bool:
+        import torch
+        lo = self.raw[:GUARD_BYTES]
+        hi = self.raw[GUARD_BYTES + self.nbytes:]
+        return bool(torch.all(lo == GUARD_FILL).item() and torch.all(hi == GUARD_FILL).item())

@@ -69,3 +69,16 @@ def test_token_rates():
     # partial lines (a leg switched off) keep working
     for partial in ({"ms_per_step": None, "config": {}, "decode": None}, {"decode": {"ms_per_step": 1.0}}, {}):
         bench.add_token_rates(partial, 1)
+
+
+def test_varlen_flops_sum_per_sequence():
+    # each packed sequence attends only to itself: 4 H L^2 D per sequence, by brute-force pair count
+    lengths, H, D = [3, 1, 7, 0, 5], 2, 64
+    pairs = sum(sum(1 for i in range(L) for j in range(L)) for L in lengths)
+    assert bench.varlen_flops(lengths, H, D) == 4 * H * D * pairs
+    assert bench.varlen_flops(lengths, H, D, causal=True) == 2 * H * D * pairs
+    # the varlen workload's figure from its seeded lengths (about 3.9e11)
+    import seeded_inputs as si
+    c = si.CONFIGS["varlen"]
+    f = bench.varlen_flops(si.varlen_lengths(c["seed"], c["nseq"], c["len_lo"], c["len_hi"]), c["H"], c["D"])
+    assert 2e11 < f < 6e11
