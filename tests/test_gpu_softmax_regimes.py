@@ -12,8 +12,8 @@ never make the kernels rescale.  Here the inputs are built so that they must:
     key axis (seeded_inputs.key_ramp), so each row's max climbs block after block -- by more than
     the kernels' deferred-rescale threshold (2^8) many times per row, or, with a gentle ramp, in
     steps below it so the stale max is carried across several blocks;
-  * large scores: fp16 / bf16 Q and K with standard deviation 3 and scale 0.5, so the largest score
-    of a row is far above 88.7, where exp overflows even in fp32.
+  * large scores: fp16 Q and K with standard deviation 3 and scale 0.5, so the largest score of a
+    row is far above 88.7, where exp overflows even in fp32.
 Every case is compared with the fp64 oracle element by element (|dO| <= 1e-2, |dLSE| <= 1e-3), and
 each rising-score case first checks on the CPU that its inputs really raise the max as intended.
 """
@@ -147,8 +147,11 @@ LARGE = [
     (1, 512, 2, 64, "fp16", False, "fp32"),
     (1, 512, 2, 64, "fp16", True, "fp16"),
     (1, 384, 2, 128, "fp16", True, "fp32"),
-    (1, 384, 2, 128, "bf16", False, "fp32"),
+    (1, 384, 2, 128, "fp16", False, "fp32"),
 ]
+# bf16 is left out on purpose: with nearly one-hot rows the rounding of P to bf16 before the P*V
+# product (relative 2^-9) alone moves O by up to 2^-9 * max|V| ~ 1e-2 for N(0,1) values, the size of
+# the tolerance; fp16 P (relative 2^-12) keeps that error at ~1e-3, and fp16 is the pages' case.
 
 
 @pytest.mark.parametrize("case", LARGE, ids=[f"n{c[1]}d{c[3]}{c[4]}{'c' if c[5] else 'n'}{c[6]}" for c in LARGE])
