@@ -4,11 +4,14 @@ Usage: ``python -m exact_tiled_attention_47_b200.build [-v]``.  Each ``csrc/*.cu
 object under ``_build/`` (skipped when up to date) and the objects are linked into
 ``exact_tiled_attention_47_b200/lib/libfa_sm100.so`` with the CUDA runtime linked statically, so the
 library needs no CUDA shared library at load time (the driver is reached through the runtime).
+Kernels that re-split registers between warpgroups (setmaxnreg) are checked against the ptxas report:
+the build fails unless they got exactly the register count their source plans for.
 """
 from __future__ import annotations
 
 import argparse
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -44,6 +47,50 @@ def _headers():
     return hs
 
 
+# Kernels whose warpgroups re-split their registers with setmaxnreg: the split only works when the
+# kernel is launched with exactly the register count the source plans for (kLaunchRegs), so the
+# build fails if ptxas allocated anything else or spilled.
+REGISTER_PLANNED = {"fa_prefill_sm100.cu": ("fa_fwd_kernel", "kLaunchRegs")}
+
+
+def ptxas_kernels(report: str):
+    """{mangled entry name: (registers, spill bytes)} from a ``-Xptxas -v`` report."""
+    out, cur = {}, None
+    for line in report.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur = m.group(1)
+            out[cur] = [None, 0]
+            continue
+        if cur is None:
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m:
+            out[cur][1] = int(m.group(1)) + int(m.group(2))
+        m = re.search(r"Used (\d+) registers", line)
+        if m:
+            out[cur][0] = int(m.group(1))
+    return {k: tuple(v) for k, v in out.items()}
+
+
+def check_planned_registers(src_name: str, source: str, report: str) -> None:
+    """Raise RuntimeError unless every planned kernel of the file got exactly its planned registers."""
+    if src_name not in REGISTER_PLANNED:
+        return
+    kernel, const = REGISTER_PLANNED[src_name]
+    m = re.search(r"constexpr int " + const + r" = (\d+);", source)
+    if not m:
+        raise RuntimeError(f"{src_name}: no '{const}' constant found")
+    planned = int(m.group(1))
+    found = {k: v for k, v in ptxas_kernels(report).items() if kernel in k}
+    if not found:
+        raise RuntimeError(f"{src_name}: ptxas reported no {kernel} instantiation")
+    bad = {k: v for k, v in found.items() if v[0] != planned or v[1] != 0}
+    if bad:
+        raise RuntimeError(f"{src_name}: {kernel} must use exactly {planned} registers without spills "
+                           f"(setmaxnreg split); ptxas gave {sorted(set(bad.values()))}")
+
+
 def _stale(target: str, deps) -> bool:
     if not os.path.exists(target):
         return True
@@ -64,19 +111,27 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [cc] + ARCH + CFLAGS + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", src, "-o", obj]
-            jobs.append(cmd)
+            planned = os.path.basename(src) in REGISTER_PLANNED
+            cmd = [cc] + ARCH + CFLAGS + (["-Xptxas", "-v"] if (ptxas_info or planned) else []) + ["-c", src, "-o", obj]
+            jobs.append((src, obj, cmd))
 
-    def run(cmd):
+    def run(job):
+        src, obj, cmd = job
         r = subprocess.run(cmd, capture_output=True, text=True)
-        return cmd, r
+        return src, obj, cmd, r
 
     with ThreadPoolExecutor(max(1, min(len(jobs), os.cpu_count() or 1)) or 1) as ex:
-        for cmd, r in ex.map(run, jobs):
+        for src, obj, cmd, r in ex.map(run, jobs):
             if verbose or ptxas_info:
                 sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+            try:
+                with open(src) as fh:
+                    check_planned_registers(os.path.basename(src), fh.read(), r.stdout + r.stderr)
+            except RuntimeError:
+                os.remove(obj)  # never link (or count as up to date) an object that failed the check
+                raise
     if force or jobs or _stale(LIB, objs):
         cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)

@@ -4,6 +4,8 @@
 // element types, head dimension, shapes and scale, alignment, workspace, then the device.  Kernels
 // report failures they detect (a bounded wait that ran out, an inconsistent cu_seqlens) through a
 // per-device status word read by fa_device_status().
+#include <cuda.h>
+
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -18,10 +20,38 @@ __device__ int g_status_word = 0;
 
 constexpr int kMaxDevices = 64;
 int g_device_ok[kMaxDevices];      // 0 unknown, 1 sm_100, -1 other
-int* g_status_ptr[kMaxDevices];
 std::mutex g_mu;
+PerContext<int*> g_status_ptr;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
 }  // namespace
+
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -47,18 +77,18 @@ int check_device(int* dev_out) {
 }
 
 int* device_status_ptr() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
+  int* out = nullptr;
+  const int e = g_status_ptr.get(&out, [](int** v) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+    const cudaError_t r = cudaGetSymbolAddress(&p, g_status_word);
+    if (r != cudaSuccess || p == nullptr) {
       cudaGetLastError();
-      return nullptr;
+      return static_cast<int>(r != cudaSuccess ? r : cudaErrorInvalidSymbol);
     }
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_status_ptr[dev];
+    *v = static_cast<int*>(p);
+    return 0;
+  });
+  return e == 0 ? out : nullptr;
 }
 
 }  // namespace fa
@@ -167,28 +197,37 @@ size_t fa_decode_workspace_bytes(int B, int H, int D, int num_splits) {
 
 namespace {
 
-int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
-                int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k, void* workspace,
-                size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype, int key_offset = 0,
-                int Nk_total = 0) {
+// Argument checks of every split-KV decode entry point, in the boundary's fixed order.  The
+// workspace is either the caller's (ws != nullptr required, at least ws_bytes, 16-byte aligned) or
+// the library's fixed scratch array (fixed_ws: only its capacity ws_bytes is checked).
+int decode_check(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
+                 int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k, const void* ws,
+                 size_t ws_bytes, bool fixed_ws, int in_dtype, int o_dtype, int key_offset, int Nk_total) {
   if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_NULL;
   if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
   if (o_dtype != in_dtype && o_dtype != FA_FP32) return FA_ERR_DTYPE;
   if (D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || Nk < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_SHAPE;
-  if (Nk_total == 0) Nk_total = Nk;
   if (key_offset < 0 || static_cast<int64_t>(key_offset) + Nk > Nk_total) return FA_ERR_SHAPE;
   if (num_splits < 1 || num_splits > 128) return FA_ERR_SHAPE;
   if (static_cast<int64_t>(B) * H > (static_cast<int64_t>(1) << 28)) return FA_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
   if (!fa::aligned(q, 16) || !fa::aligned(k_cache, 16) || !fa::aligned(v_cache, 16) || !fa::aligned(o, 16) || !fa::aligned(lse, 4))
     return FA_ERR_ALIGN;
-  if (!workspace || workspace_bytes < fa_decode_workspace_bytes(B, H, D, num_splits)) return FA_ERR_WORKSPACE;
-  if (!fa::aligned(workspace, 16)) return FA_ERR_ALIGN;
+  if ((!fixed_ws && !ws) || ws_bytes < fa_decode_workspace_bytes(B, H, D, num_splits)) return FA_ERR_WORKSPACE;
+  if (!fixed_ws && !fa::aligned(ws, 16)) return FA_ERR_ALIGN;
   if (seqlens_k && !fa::aligned(seqlens_k, 4)) return FA_ERR_ALIGN;
-  int dev = -1;
-  if (const int st = fa::check_device(&dev)) return st;
+  return FA_OK;
+}
+
+}  // namespace
+
+namespace fa {
+
+int decode_checked_launch(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
+                          int H, int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k,
+                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream) {
   int* status = fa::device_status_ptr();
   if (!status) return FA_ERR_LAUNCH;
   fa::DecodeArgs a;
@@ -198,8 +237,8 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o
   a.o = o;
   a.lse = lse;
   const size_t n = static_cast<size_t>(num_splits) * B * H;
-  a.ws_o = static_cast<float*>(workspace);
-  a.ws_lse = static_cast<float*>(workspace) + n * D;
+  a.ws_o = static_cast<float*>(ws);
+  a.ws_lse = static_cast<float*>(ws) + n * D;
   a.status = status;
   a.B = B;
   a.H = H;
@@ -213,12 +252,37 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o
   a.seqlens_k = seqlens_k;
   a.key_offset = key_offset;
   a.Nk_total = Nk_total;
-  const int e = fa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  const int e = fa::launch_decode(a, stream);
   if (e != 0) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+int decode_check_fixed(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
+                       int Nk, int D, float scale, int num_splits, size_t capacity, int in_dtype, int o_dtype) {
+  return decode_check(q, k_cache, v_cache, o, lse, B, H, H, Nk, D, scale, num_splits, nullptr, nullptr, capacity,
+                      true, in_dtype, o_dtype, 0, Nk);
+}
+
+}  // namespace fa
+
+namespace {
+
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
+                int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k, void* workspace,
+                size_t workspace_bytes, fa_stream_t stream, int in_dtype, int o_dtype, int key_offset = 0,
+                int Nk_total = 0) {
+  if (Nk_total == 0) Nk_total = Nk;
+  if (const int st = decode_check(q, k_cache, v_cache, o, lse, B, H, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                                  workspace, workspace_bytes, false, in_dtype, o_dtype, key_offset, Nk_total))
+    return st;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  return fa::decode_checked_launch(q, k_cache, v_cache, o, lse, B, H, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                                   workspace, in_dtype, o_dtype, key_offset, Nk_total,
+                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace

@@ -626,11 +626,16 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   bwd_rowterm_kernel<kFp16, D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(a.o, a.dout, a.drow,
                                                                                              a.B, a.H, a.Nq);
   auto kq = bwd_dq_kernel<D, kFp16, kOutF32>;
-  cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return static_cast<int>(e);
   auto kkv = bwd_dkdv_kernel<D, kFp16, kOutF32>;
-  e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return static_cast<int>(e);
+  // the shared-memory opt-in is a per-device (per-context) attribute: raised once
+  static PerContext<int> configured;
+  int unused = 0;
+  const int ce = configured.get(&unused, [&](int*) {
+    cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return static_cast<int>(e);
+  });
+  if (ce != 0) return ce;
   BwdParams pq = p;
   pq.g0 = a.dq;
   pq.num_tiles = (a.Nq + kBT - 1) / kBT;

@@ -638,16 +638,13 @@ int launch_mma(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
       !make_tma_map(&mv, a.v, rows, p.Hkv, D, kFp16, kMmaTileKeys))
     return static_cast<int>(cudaErrorInvalidValue);
   auto kern = decode_mma_kernel<kFp16, D, G>;
-  // the shared-memory opt-in is a per-device attribute of the function: set it once per device
-  static std::atomic<uint64_t> configured{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return static_cast<int>(cudaErrorInvalidDevice);
-  if (!((configured.load(std::memory_order_acquire) >> dev) & 1u)) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MmaCfg<D>::kSmemBytes);
-    if (e != cudaSuccess) return static_cast<int>(e);
-    configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
-  }
+  // the shared-memory opt-in is a per-device (per-context) attribute of the function: set it once
+  static PerContext<int> configured;
+  int unused = 0;
+  const int ce = configured.get(&unused, [&](int*) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MmaCfg<D>::kSmemBytes));
+  });
+  if (ce != 0) return ce;
   kern<<<dim3(p.Hkv * (p.group / G), a.S, a.B), kMmaThreads, MmaCfg<D>::kSmemBytes, stream>>>(mk, mv, p);
   return 0;
 }

@@ -3,6 +3,8 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 namespace fa {
@@ -81,8 +83,60 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 int launch_decode_merge(const MergeArgs& a, cudaStream_t stream);
 int launch_backward(const BackwardArgs& a, cudaStream_t stream);
 
+// Split-KV decode after its arguments passed the boundary's checks and the device check: launches
+// the split and combine kernels with the per-split partials in ws.  Returns an fa_status.
+int decode_checked_launch(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
+                          int H, int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k,
+                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream);
+// The boundary's decode argument checks for a workspace of fixed capacity (no caller pointer).
+int decode_check_fixed(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
+                       int Nk, int D, float scale, int num_splits, size_t capacity, int in_dtype, int o_dtype);
+
 int* device_status_ptr();  // address of this device's status word (nullptr on failure)
 int check_device(int* dev_out);  // FA_OK if the current device is sm_100, else FA_ERR_DEVICE
 bool aligned(const void* p, uintptr_t a);
+
+// Unique id of the calling thread's current CUDA context (0 if none is current or the driver cannot
+// say).  Contexts are never given the id of an earlier one, so a cached per-device value tagged
+// with it is known to be stale once the device's context was destroyed and recreated (for example
+// by cudaDeviceReset).
+unsigned long long current_context_id();
+
+// A value set up once per device and CUDA context (a symbol's device address, a function attribute
+// that was raised): make(&v) runs on the first use in a context and again whenever the current
+// context's id differs from the one recorded, and its error is returned without being cached.
+template <class T>
+class PerContext {
+ public:
+  template <class F>
+  int get(T* out, F&& make) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSlots) {
+      cudaGetLastError();
+      return static_cast<int>(cudaErrorInvalidDevice);
+    }
+    std::lock_guard<std::mutex> lk(mu_);
+    const unsigned long long id = current_context_id();
+    if (ok_[dev] && id != 0 && id == ctx_[dev]) {
+      *out = val_[dev];
+      return 0;
+    }
+    T v{};
+    const int e = make(&v);
+    if (e != 0) return e;
+    val_[dev] = v;
+    ctx_[dev] = current_context_id();  // make() has initialised the context if it was not yet
+    ok_[dev] = true;
+    *out = v;
+    return 0;
+  }
+
+ private:
+  static constexpr int kSlots = 64;
+  std::mutex mu_;
+  T val_[kSlots]{};
+  unsigned long long ctx_[kSlots]{};
+  bool ok_[kSlots]{};
+};
 
 }  // namespace fa

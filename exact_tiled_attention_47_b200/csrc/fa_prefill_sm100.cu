@@ -50,7 +50,8 @@ constexpr int kPanelBytes = kBM * 64 * 2;  // one 64-column (128-byte) swizzle p
 // Registers: launched with kLaunchRegs per thread; the two softmax warpgroups then take
 // kSoftmaxRegs and the producer/MMA warpgroup gives back down to kControlRegs.  The split must not
 // exceed the launch allocation (256 * 216 + 128 * 72 = 384 * 168), else setmaxnreg.inc would wait
-// forever; the host refuses to launch if the compiled register count differs from kLaunchRegs.
+// forever.  The build checks (ptxas report) that every instantiation is compiled to exactly
+// kLaunchRegs registers, and the host confirms it once per device before the first launch.
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 216;
 constexpr int kControlRegs = 72;
@@ -459,12 +460,19 @@ int launch_t(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
              const FwdParams& p, cudaStream_t stream) {
   auto kern = fa_fwd_kernel<D, kFp16, kOutF32>;
   const int smem = Cfg<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return static_cast<int>(e);
-  cudaFuncAttributes fattr;
-  e = cudaFuncGetAttributes(&fattr, kern);
-  if (e != cudaSuccess) return static_cast<int>(e);
-  if (fattr.numRegs != kLaunchRegs) return static_cast<int>(cudaErrorInvalidConfiguration);
+  // Once per device and context: raise the shared-memory limit and confirm the register count the
+  // build checked (the setmaxnreg split above needs exactly the launch allocation).
+  static PerContext<int> configured;
+  int unused = 0;
+  const int ce = configured.get(&unused, [&](int*) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    cudaFuncAttributes fattr;
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    return fattr.numRegs == kLaunchRegs ? 0 : static_cast<int>(cudaErrorInvalidConfiguration);
+  });
+  if (ce != 0) return ce;
   long long blocks;
   if (a.cu_seqlens == nullptr)
     blocks = static_cast<long long>(p.num_units) * a.B * a.H;

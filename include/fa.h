@@ -28,6 +28,8 @@
  *     status code is returned.  No entry point aborts, throws or prints.
  *   - Device-side failures (a bounded wait inside a kernel that ran out) are recorded in a device
  *     status word that fa_device_status() reads.
+ *   - Per-device set-up (the status word's address, raised shared-memory limits) is done once per
+ *     CUDA context and redone when the device's context changes (for example after cudaDeviceReset).
  */
 #ifndef FA_SM100_H
 #define FA_SM100_H
@@ -249,7 +251,11 @@ int fa_decode_merge(const float* parts, int R, int B, int H, int D, void* o, flo
  *   - Returns FA_ERR_WORKSPACE, without launching, when fa_decode_workspace_bytes(B, H, D,
  *     num_splits) exceeds FA_NOALLOC_SCRATCH_BYTES.
  *   - The first call on a device looks up the array's device address (with that device current)
- *     and caches it; make that first call before any stream capture.
+ *     and caches it for that device's CUDA context; make that first call before any stream
+ *     capture.  After the context is destroyed and recreated (cudaDeviceReset), the next call looks
+ *     the address up again.
+ *   - Its argument checks are those of fa_decode_splitkv, in the same order, with the fixed array's
+ *     capacity in place of workspace_bytes.
  *   - Every call on a device shares the one array.  Nothing in it needs clearing between calls, but
  *     calls whose kernels may overlap on the GPU (unordered streams) race on it: order them.
  *   - Calls no allocating routine (no cudaMalloc / cudaFree).
