@@ -11,17 +11,18 @@ from __future__ import annotations
 import ctypes
 import math
 
-from ._lib import LIB_PATH, LibraryMissing, SIGNATURES, load
+from ._lib import DEBUG_LIB_PATH, LIB_PATH, LibraryMissing, SIGNATURES, load
 
 FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 (FA_OK, FA_ERR_NULL, FA_ERR_DTYPE, FA_ERR_HEADDIM, FA_ERR_SHAPE, FA_ERR_ALIGN, FA_ERR_CU_SEQLENS,
- FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT) = range(11)
+ FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT, FA_ERR_BOUNDS) = range(12)
+FA_BUILD_DEBUG = 1
 
 __all__ = [
     "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
-    "fa_device_status", "fa_abi_version", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
+    "fa_device_status", "fa_abi_version", "fa_build_flags", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "decode_sharded", "shard_range", "attention", "decode", "FAError", "LibraryMissing",
-    "LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32",
+    "LIB_PATH", "DEBUG_LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32", "FA_BUILD_DEBUG",
 ]
 
 
@@ -207,6 +208,10 @@ def fa_selftest_wait_timeout(stream=None):
 
 def fa_abi_version() -> int:
     return int(load().fa_abi_version())
+
+
+def fa_build_flags() -> int:
+    return int(load().fa_build_flags())
 
 
 # ------------------------------------------------------------------------------------------------

@@ -9,6 +9,8 @@ import os
 import threading
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa_sm100.so")
+# The same entry points built with index checks (FA_DEBUG); loaded only when asked for by path.
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa_sm100_debug.so")
 
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -30,6 +32,7 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_device_status": (_I, [ctypes.POINTER(_I), _I]),
     "fa_abi_version": (_I, []),
+    "fa_build_flags": (_I, []),
     "fa_selftest_wait_timeout": (_I, [ctypes.POINTER(_I), _P]),
 }
 

@@ -24,6 +24,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libfa_sm100.so")
+DEBUG_LIB = os.path.join(LIBDIR, "libfa_sm100_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -98,9 +99,16 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) -> str:
-    """Compile and link; returns the library path.  Raises RuntimeError on a compiler error."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False, debug: bool = False) -> str:
+    """Compile and link; returns the library path.  Raises RuntimeError on a compiler error.
+
+    ``debug`` builds ``libfa_sm100_debug.so`` instead: the same sources with ``-DFA_DEBUG`` (index
+    checks on every plain global access, reported as FA_ERR_BOUNDS; the prefill walks every key
+    block of a causal row instead of skipping the fully masked ones), objects under ``_build/debug``.
+    """
+    bdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib_path = DEBUG_LIB if debug else LIB
+    os.makedirs(bdir, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     cc = nvcc()
     headers = _headers()
@@ -108,11 +116,12 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
     objs = []
     jobs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
             planned = os.path.basename(src) in REGISTER_PLANNED
-            cmd = [cc] + ARCH + CFLAGS + (["-Xptxas", "-v"] if (ptxas_info or planned) else []) + ["-c", src, "-o", obj]
+            cmd = ([cc] + ARCH + CFLAGS + (["-DFA_DEBUG"] if debug else []) +
+                   (["-Xptxas", "-v"] if (ptxas_info or planned) else []) + ["-c", src, "-o", obj])
             jobs.append((src, obj, cmd))
 
     def run(job):
@@ -132,14 +141,14 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
             except RuntimeError:
                 os.remove(obj)  # never link (or count as up to date) an object that failed the check
                 raise
-    if force or jobs or _stale(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+    if force or jobs or _stale(lib_path, objs):
+        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", lib_path] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if verbose:
             sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
-    return LIB
+    return lib_path
 
 
 if __name__ == "__main__":
@@ -147,5 +156,6 @@ if __name__ == "__main__":
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers/spills per kernel")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build the index-checking debug library instead")
     a = ap.parse_args()
-    print(build(a.verbose, a.ptxas_info, a.force))
+    print(build(a.verbose, a.ptxas_info, a.force, a.debug))

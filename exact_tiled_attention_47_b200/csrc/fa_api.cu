@@ -97,6 +97,14 @@ extern "C" {
 
 int fa_abi_version(void) { return 1; }
 
+int fa_build_flags(void) {
+#ifdef FA_DEBUG
+  return FA_BUILD_DEBUG;
+#else
+  return 0;
+#endif
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "ok";
@@ -110,6 +118,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE: return "no usable sm_100 (B200) CUDA device";
     case FA_ERR_LAUNCH: return "CUDA launch or driver call failed";
     case FA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case FA_ERR_BOUNDS: return "an index check of the debug build caught an access outside its buffer";
     default: return "unknown status";
   }
 }
@@ -342,6 +351,8 @@ int fa_decode_merge(const float* parts, int R, int B, int H, int D, void* o, flo
   a.lse = lse;
   a.o_fp16 = o_dtype == FA_FP16;
   a.o_fp32 = o_dtype == FA_FP32;
+  a.status = fa::device_status_ptr();
+  if (!a.status) return FA_ERR_LAUNCH;
   if (fa::launch_decode_merge(a, reinterpret_cast<cudaStream_t>(stream)) != 0) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;

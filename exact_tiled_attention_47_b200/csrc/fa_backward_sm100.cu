@@ -63,6 +63,7 @@ struct BwdParams {
   const float* drow;  // [B, H, Nq]
   void* g0;           // dq (dq kernel) or dk (dkdv kernel)
   void* g1;           // dv (dkdv kernel)
+  long long g0_n, g1_n;  // elements of g0 and g1 (bounds of the debug index checks)
   int* status;
   int B, H, Nq, Nk;
   int num_tiles;  // query tiles (dq) or key tiles (dkdv) per (b, h)
@@ -86,9 +87,11 @@ static_assert(sizeof(BwdBars) <= 256, "barrier block too large");
 
 template <bool kFp16, int D>
 __global__ void __launch_bounds__(256) bwd_rowterm_kernel(const void* o, const void* dout, float* drow, int B,
-                                                          int H, int N) {
+                                                          int H, int N, int* status) {
   const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b, i, h) row
-  if (r >= static_cast<long long>(B) * N * H) return;
+  const long long rows = static_cast<long long>(B) * N * H;
+  if (r >= rows) return;
+  if (!idx_ok(status, r * D, D, rows * D)) return;
   const uint4* a = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(o) + r * D);
   const uint4* g = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(dout) + r * D);
   float acc = 0.f;
@@ -106,7 +109,8 @@ __global__ void __launch_bounds__(256) bwd_rowterm_kernel(const void* o, const v
   const long long bi = r / H;
   const int i = static_cast<int>(bi % N);
   const int b = static_cast<int>(bi / N);
-  drow[(static_cast<size_t>(b) * H + h) * N + i] = acc;
+  const size_t di = (static_cast<size_t>(b) * H + h) * N + i;
+  if (idx_ok(status, di, 1, rows)) drow[di] = acc;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -172,7 +176,8 @@ constexpr uint32_t kHalfRowOff = kHalf * 128;
 // Columns [32 * ch_lo, 32 * ch_hi) of the row.
 template <int D, bool kFp16, bool kOutF32>
 __device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint32_t taddr, float mul, bool store,
-                                               int ch_lo = 0, int ch_hi = D / 32) {
+                                               int* status, long long out_n, int ch_lo = 0, int ch_hi = D / 32) {
+  if (store) store = idx_ok(status, row_elem, D, out_n);
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
     if (ch < ch_lo || ch >= ch_hi) continue;
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qi = m0 + warp * 32 + lane;
       if (qi < Lq) {
         const size_t row = ((static_cast<size_t>(b) * Lq + qi) * p.H + h) * D;
-        for (int d = 0; d < D; ++d) {
+        for (int d = 0; d < D && idx_ok(p.status, row, D, p.g0_n); ++d) {
           if constexpr (kOutF32) static_cast<float*>(p.g0)[row + d] = 0.f;
           else static_cast<uint16_t*>(p.g0)[row + d] = 0;
         }
@@ -351,10 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;
     const int tile_lim = p.causal ? min(Lk, m0 + 1 + diag) : Lk;
     const size_t stat = (static_cast<size_t>(b) * p.H + h) * Lq + min(qi, Lq - 1);
-    const float lse = p.lse[stat];
+    const bool stat_in = idx_ok(p.status, stat, 1, static_cast<long long>(p.B) * p.H * Lq);
+    const float lse = stat_in ? p.lse[stat] : -INFINITY;
     // rows without keys (LSE = -inf) and rows past the end get P = 0
     const float lse2 = (qi < Lq && lse != -INFINITY) ? lse * kLog2e : INFINITY;
-    const float dr = (qi < Lq) ? p.drow[stat] : 0.f;
+    const float dr = (qi < Lq && stat_in) ? p.drow[stat] : 0.f;
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -400,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const size_t row = (static_cast<size_t>(b) * Lq + min(qi, Lq - 1)) * p.H + h;
       // the two halves of warps store the two halves of the row
-      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, hh * D / 64,
-                                        (hh + 1) * D / 64);
+      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, p.status, p.g0_n,
+                                        hh * D / 64, (hh + 1) * D / 64);
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -441,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kj = n0 + warp * 32 + lane;
       if (kj < Lk) {
         const size_t row = ((static_cast<size_t>(b) * Lk + kj) * p.H + h) * D;
-        for (int d = 0; d < D; ++d) {
+        for (int d = 0; d < D && idx_ok(p.status, row, D, p.g0_n) && idx_ok(p.status, row, D, p.g1_n); ++d) {
           if constexpr (kOutF32) {
             static_cast<float*>(p.g0)[row + d] = 0.f;
             static_cast<float*>(p.g1)[row + d] = 0.f;
@@ -490,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int qi = i * kBT + lane + 32 * u;
-        const bool in = qi < Lq;
+        const bool in = qi < Lq && idx_ok(p.status, base + qi, 1, static_cast<long long>(p.B) * p.H * Lq);
         lv[u] = in ? p.lse[base + qi] : -INFINITY;
         dv[u] = in ? p.drow[base + qi] : 0.f;
       }
@@ -612,8 +618,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const size_t row = ((static_cast<size_t>(b) * Lk + min(kj, Lk - 1)) * p.H + h) * D;
-      if (hh == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk);  // dV
-      else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk);  // dK
+      if (hh == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk, p.status, p.g1_n);  // dV
+      else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk, p.status, p.g0_n);  // dK
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -624,7 +630,7 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   const int smem = BwdCfg<D>::kSmemBytes;
   const size_t rows = static_cast<size_t>(a.B) * a.Nq * a.H;
   bwd_rowterm_kernel<kFp16, D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(a.o, a.dout, a.drow,
-                                                                                             a.B, a.H, a.Nq);
+                                                                                             a.B, a.H, a.Nq, a.status);
   auto kq = bwd_dq_kernel<D, kFp16, kOutF32>;
   auto kkv = bwd_dkdv_kernel<D, kFp16, kOutF32>;
   // the shared-memory opt-in is a per-device (per-context) attribute: raised once
@@ -638,11 +644,13 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   if (ce != 0) return ce;
   BwdParams pq = p;
   pq.g0 = a.dq;
+  pq.g0_n = static_cast<long long>(a.B) * a.Nq * a.H * D;
   pq.num_tiles = (a.Nq + kBT - 1) / kBT;
   kq<<<static_cast<unsigned>(pq.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pq);
   BwdParams pk = p;
   pk.g0 = a.dk;
   pk.g1 = a.dv;
+  pk.g0_n = pk.g1_n = static_cast<long long>(a.B) * a.Nk * a.H * D;
   pk.num_tiles = (a.Nk + kBT - 1) / kBT;
   kkv<<<static_cast<unsigned>(pk.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pk);
   return static_cast<int>(cudaGetLastError());
@@ -661,6 +669,7 @@ int launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   p.lse = a.lse;
   p.drow = a.drow;
   p.g0 = p.g1 = nullptr;
+  p.g0_n = p.g1_n = 0;
   p.status = a.status;
   p.B = a.B;
   p.H = a.H;

@@ -54,6 +54,16 @@ struct DecParams {
   float scale_log2;
 };
 
+// Elements of the buffers a decode kernel touches with plain loads and stores (debug index checks).
+__device__ __forceinline__ long long q_elems(const DecParams& p, int D) { return static_cast<long long>(p.B) * p.H * D; }
+__device__ __forceinline__ long long kv_elems(const DecParams& p, int D) {
+  return static_cast<long long>(p.B) * p.Nk * p.Hkv * D;
+}
+__device__ __forceinline__ long long ws_o_elems(const DecParams& p, int D) {
+  return static_cast<long long>(p.B) * p.H * p.S * D;
+}
+__device__ __forceinline__ long long ws_l_elems(const DecParams& p) { return static_cast<long long>(p.B) * p.H * p.S; }
+
 // Partial results to merge: partial t of output row r (= b * H + h) has its normalised output at
 // po + r * o_row + t * o_part (D floats) and its natural-log LSE at pl + r * l_row + t * l_part.
 struct CombParams {
@@ -63,6 +73,8 @@ struct CombParams {
   int T, rows;
   void* o;
   float* lse;
+  long long po_n, pl_n;  // floats readable from po and from pl (bounds of the debug index checks)
+  int* status;
 };
 
 template <bool kFp16>
@@ -112,8 +124,9 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   if (lo >= hi) {  // a split past the end of the valid cache: empty partials
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      for (int d = tid; d < D; d += kDecThreads) ws_o(g)[d] = 0.f;
-      if (tid == 0) *ws_l(g) = -INFINITY;
+      for (int d = tid; d < D; d += kDecThreads)
+        if (idx_ok(p.status, ws_o(g) + d - p.ws_o, 1, ws_o_elems(p, D))) ws_o(g)[d] = 0.f;
+      if (tid == 0 && idx_ok(p.status, ws_l(g) - p.ws_lse, 1, ws_l_elems(p))) *ws_l(g) = -INFINITY;
     }
     return;
   }
@@ -121,7 +134,13 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   float qf[G][8];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    load8_stream<kFp16>(static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.H + hq0 + g) * D + c * 8, qf[g]);
+    const size_t qoff = (static_cast<size_t>(b) * p.H + hq0 + g) * D + c * 8;
+    if (idx_ok(p.status, qoff, 8, q_elems(p, D))) {
+      load8_stream<kFp16>(static_cast<const T*>(p.q) + qoff, qf[g]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[g][e] = 0.f;
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;  // scores come out in log2 units
   }
@@ -147,7 +166,8 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        if (j < n) {
+        if (j < n && idx_ok(p.status, kb + static_cast<size_t>(c0 + j) * rs - static_cast<const T*>(p.k), 8,
+                            kv_elems(p, D))) {
           load8_stream<kFp16>(kb + static_cast<size_t>(c0 + j) * rs, kf[u]);
         } else {
 #pragma unroll
@@ -194,7 +214,8 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        if (j < n) {
+        if (j < n && idx_ok(p.status, vb + static_cast<size_t>(c0 + j) * rs - static_cast<const T*>(p.v), 8,
+                            kv_elems(p, D))) {
           load8_stream<kFp16>(vb + static_cast<size_t>(c0 + j) * rs, vf[u]);
         } else {
 #pragma unroll
@@ -240,8 +261,9 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
     const float inv_l = 1.f / l;
     float* wo = ws_o(g);
     for (int d = tid; d < D; d += kDecThreads)
-      wo[d] = (red_acc[0][g][d] + red_acc[1][g][d] + red_acc[2][g][d] + red_acc[3][g][d]) * inv_l;
-    if (tid == 0) *ws_l(g) = (m_run[g] + lg2(l)) * kLn2;
+      if (idx_ok(p.status, wo + d - p.ws_o, 1, ws_o_elems(p, D)))
+        wo[d] = (red_acc[0][g][d] + red_acc[1][g][d] + red_acc[2][g][d] + red_acc[3][g][d]) * inv_l;
+    if (tid == 0 && idx_ok(p.status, ws_l(g) - p.ws_lse, 1, ws_l_elems(p))) *ws_l(g) = (m_run[g] + lg2(l)) * kLn2;
   }
 }
 
@@ -361,8 +383,9 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
   auto ws_o = [&](int g) { return p.ws_o + ((static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s) * D; };
   auto ws_l = [&](int g) { return p.ws_lse + (static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s; };
   if (lo >= hi) {  // uniform over the CTA: empty partials
-    for (int i = tid; i < G * D; i += kMmaThreads) ws_o(i / D)[i % D] = 0.f;
-    if (tid < G) *ws_l(tid) = -INFINITY;
+    for (int i = tid; i < G * D; i += kMmaThreads)
+      if (idx_ok(p.status, ws_o(i / D) + i % D - p.ws_o, 1, ws_o_elems(p, D))) ws_o(i / D)[i % D] = 0.f;
+    if (tid < G && idx_ok(p.status, ws_l(tid) - p.ws_lse, 1, ws_l_elems(p))) *ws_l(tid) = -INFINITY;
     return;
   }
   const int n_tiles = (hi - lo + kMmaTileKeys - 1) / kMmaTileKeys;
@@ -414,13 +437,14 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     {
       const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
       const size_t qrow = (static_cast<size_t>(b) * p.H + hq0) * D;
+      const bool q_in = idx_ok(p.status, qrow, static_cast<long long>(G) * D, q_elems(p, D));
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         const int c = ks * 16 + 2 * tg;
-        qa[ks][0] = (g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c) / 2) : 0u;
-        qa[ks][2] = (g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c + 8) / 2) : 0u;
-        qa[ks][1] = (kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c) / 2) : 0u;
-        qa[ks][3] = (kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c + 8) / 2) : 0u;
+        qa[ks][0] = (q_in && g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c) / 2) : 0u;
+        qa[ks][2] = (q_in && g < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g) * D + c + 8) / 2) : 0u;
+        qa[ks][1] = (q_in && kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c) / 2) : 0u;
+        qa[ks][3] = (q_in && kHi && g + 8 < G) ? __ldg(q32 + (qrow + static_cast<size_t>(g + 8) * D + c + 8) / 2) : 0u;
       }
     }
 #pragma unroll
@@ -557,8 +581,9 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
         acc += e * red_o[(w * G + h) * D + d];
       }
     }
-    ws_o(h)[d] = (M > -INFINITY) ? acc / l : 0.f;
-    if (d == 0) *ws_l(h) = (M > -INFINITY) ? (M + lg2(l)) * kLn2 : -INFINITY;
+    if (idx_ok(p.status, ws_o(h) + d - p.ws_o, 1, ws_o_elems(p, D))) ws_o(h)[d] = (M > -INFINITY) ? acc / l : 0.f;
+    if (d == 0 && idx_ok(p.status, ws_l(h) - p.ws_lse, 1, ws_l_elems(p)))
+      *ws_l(h) = (M > -INFINITY) ? (M + lg2(l)) * kLn2 : -INFINITY;
   }
 }
 
@@ -570,6 +595,13 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const CombParams p)
   if (bh >= p.rows) return;
   const float* wl = p.pl + static_cast<long long>(bh) * p.l_row;
   const float* wo = p.po + static_cast<long long>(bh) * p.o_row;
+#ifdef FA_DEBUG
+  // every partial this row reads must lie inside the partial buffers (warp-uniform)
+  if (!idx_ok(p.status, wl - p.pl, static_cast<long long>(p.T - 1) * p.l_part + 1, p.pl_n) ||
+      !idx_ok(p.status, wo - p.po, static_cast<long long>(p.T - 1) * p.o_part + D, p.po_n) ||
+      !idx_ok(p.status, static_cast<long long>(bh) * D, D, static_cast<long long>(p.rows) * D))
+    return;
+#endif
 
   float mx = -INFINITY;
   for (int t = lane; t < p.T; t += 32) mx = fmaxf(mx, wl[t * p.l_part] * kLog2e);
@@ -675,6 +707,9 @@ int launch_decode_t(const DecodeArgs& a, const DecParams& p, cudaStream_t stream
   c.rows = a.B * a.H;
   c.o = p.o;
   c.lse = p.lse;
+  c.po_n = static_cast<long long>(a.B) * a.H * p.S * D;
+  c.pl_n = static_cast<long long>(a.B) * a.H * p.S;
+  c.status = p.status;
   launch_combine<kFp16, D>(c, a.o_fp32, stream);
   return static_cast<int>(cudaGetLastError());
 }
@@ -710,6 +745,9 @@ int launch_decode_merge(const MergeArgs& a, cudaStream_t stream) {
   c.rows = static_cast<int>(rows);
   c.o = a.o;
   c.lse = a.lse;
+  c.po_n = static_cast<long long>(a.R) * a.part_floats;
+  c.pl_n = c.po_n - rows * a.D;
+  c.status = a.status;
   if (a.D == 64) {
     if (a.o_fp16) launch_combine<true, 64>(c, a.o_fp32, stream);
     else launch_combine<false, 64>(c, a.o_fp32, stream);

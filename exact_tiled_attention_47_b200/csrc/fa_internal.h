@@ -56,6 +56,7 @@ struct MergeArgs {
   float* lse;
   int o_fp16;  // 16-bit output: fp16 (1) or bf16 (0); ignored with o_fp32
   int o_fp32;
+  int* status = nullptr;  // device status word (debug index checks)
 };
 
 struct BackwardArgs {

@@ -82,10 +82,27 @@ __device__ void find_varlen_unit(const FwdParams& p, int slot, int lane, int& ou
   out_unit = fm;
 }
 
+// Elements of the O and LSE buffers (the bounds of the debug build's index checks).
+template <int D>
+__device__ __forceinline__ long long o_elems(const FwdParams& p) {
+  return static_cast<long long>(p.cu == nullptr ? p.B : 1) * p.Nq * p.H * D;
+}
+__device__ __forceinline__ long long lse_elems(const FwdParams& p) {
+  return static_cast<long long>(p.cu == nullptr ? p.B : 1) * p.H * p.Nq;
+}
+
+// Index of a row's LSE: [B, H, Nq] dense, [H, total] packed varlen.
+__device__ __forceinline__ size_t lse_index(const FwdParams& p, int b, int h, int q_row0, int qi) {
+  return (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
+                           : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
+}
+
 // O and LSE of a row that sees no key at all.
 template <int D, bool kOutF32>
 __device__ void write_empty_row(const FwdParams& p, int b, int h, int q_row0, int qi) {
   const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
+  const size_t li0 = lse_index(p, b, h, q_row0, qi);
+  if (!idx_ok(p.status, orow, D, o_elems<D>(p)) || !idx_ok(p.status, li0, 1, lse_elems(p))) return;
   if constexpr (kOutF32) {
     float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow);
     for (int d = 0; d < D / 4; ++d) out[d] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -93,9 +110,7 @@ __device__ void write_empty_row(const FwdParams& p, int b, int h, int q_row0, in
     uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow);
     for (int d = 0; d < D / 8; ++d) out[d] = make_uint4(0, 0, 0, 0);
   }
-  const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
-                                      : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
-  p.lse[li] = -INFINITY;
+  p.lse[li0] = -INFINITY;
 }
 
 // P for 32 score columns (chunk ch of the row): x = s * scale * log2(e) - m, p = 2^x (on the MUFU
@@ -152,6 +167,9 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_taddr, 
   const bool empty = (m_run == -INFINITY);
   const float inv_l = empty ? 0.f : 1.f / l_run;
   const size_t orow = (static_cast<size_t>(q_row0 + qi) * p.H + h) * D;
+#ifdef FA_DEBUG
+  if (store) store = idx_ok(p.status, orow, D, o_elems<D>(p)) && idx_ok(p.status, lse_index(p, b, h, q_row0, qi), 1, lse_elems(p));
+#endif
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
     uint32_t orr[32];
@@ -174,11 +192,7 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_taddr, 
       }
     }
   }
-  if (store) {
-    const size_t li = (p.cu == nullptr) ? (static_cast<size_t>(b) * p.H + h) * p.Nq + qi
-                                        : static_cast<size_t>(h) * p.Nq + q_row0 + qi;
-    p.lse[li] = empty ? -INFINITY : (m_run + lg2(l_run)) * kLn2;
-  }
+  if (store) p.lse[lse_index(p, b, h, q_row0, qi)] = empty ? -INFINITY : (m_run + lg2(l_run)) * kLn2;
 }
 
 // 3-D TMA map over a [rows, H, D] 16-bit tensor: box = 64 columns x 1 head x box_rows rows, 128-byte

@@ -58,7 +58,10 @@ constexpr int kControlRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
 // Of every kEmuEvery column pairs of exponentials, kEmuPairs run on the FMA pipe (measured best of
 // 0..3 for both head dims).
-constexpr int kEmuPairs = 1;
+#ifndef FA_EMU_PAIRS
+#define FA_EMU_PAIRS 1
+#endif
+constexpr int kEmuPairs = FA_EMU_PAIRS;
 
 template <int D>
 struct Cfg {
@@ -162,7 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto blocks_of = [&](int t) {
     const int first = m0 + t * kBM;
     int kv_end = Lk;
+#ifndef FA_DEBUG  // the debug build walks every key block and lets the mask zero the invisible ones
     if (p.causal) kv_end = min(Lk, max(p.prefix, first + kBM + diag));
+#endif
     return (first < Lq && kv_end > 0) ? (kv_end + kBN - 1) / kBN : 0;
   };
   const int n_kv0 = blocks_of(0), n_kv1 = blocks_of(1);

@@ -33,6 +33,27 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+constexpr int kStatusBounds = 11;  // FA_ERR_BOUNDS
+
+// Index check of a plain global access (one that no TMA descriptor bounds): elements
+// [first, first + count) of a buffer of n elements.  Debug builds (FA_DEBUG) record FA_ERR_BOUNDS in
+// the status word and return false when the range leaves the buffer, so the caller skips the access;
+// release builds compile the check away.
+__device__ __forceinline__ bool idx_ok(int* status, long long first, long long count, long long n) {
+#ifdef FA_DEBUG
+  if (first < 0 || count < 0 || first + count > n) {
+    record_status(status, kStatusBounds);
+    return false;
+  }
+#else
+  (void)status;
+  (void)first;
+  (void)count;
+  (void)n;
+#endif
+  return true;
+}
+
 // ------------------------------------------------------------------------------------------------
 // mbarrier
 

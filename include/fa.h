@@ -56,7 +56,9 @@ typedef enum {
   FA_ERR_WORKSPACE = 7,   /* decode workspace missing or smaller than required                */
   FA_ERR_DEVICE = 8,      /* no CUDA device, or the current device is not sm_100             */
   FA_ERR_LAUNCH = 9,      /* a CUDA launch or driver call failed                              */
-  FA_ERR_TIMEOUT = 10     /* a bounded wait inside a kernel ran out (device-detected)         */
+  FA_ERR_TIMEOUT = 10,    /* a bounded wait inside a kernel ran out (device-detected)         */
+  FA_ERR_BOUNDS = 11      /* debug builds only: an index check caught an access outside its
+                             buffer (device-detected; the access was skipped)                  */
 } fa_status;
 
 /*
@@ -289,6 +291,18 @@ const char* fa_status_string(int status);
  * FA_ERR_LAUNCH.
  */
 int fa_device_status(int* status_out, int clear);
+
+/*
+ * fa_build_flags -- how this library was built.  Bit 0 (FA_BUILD_DEBUG): a debug build
+ * (libfa_sm100_debug.so): every plain global load and store of the kernels (those no TMA descriptor
+ * bounds) checks its index against its buffer and, when it would leave it, skips the access and
+ * records FA_ERR_BOUNDS in the device status word; the prefill kernel also walks every key block of
+ * a causal or prefix-masked row instead of stopping after the last visible one, masking the rest
+ * (the results are the same bit for bit).  The pages have no counterpart: this is test equipment
+ * standing in for a memory checker.  Never fails.
+ */
+#define FA_BUILD_DEBUG 1
+int fa_build_flags(void);
 
 /* fa_abi_version -- version of this interface (incremented on any signature change). */
 int fa_abi_version(void);

@@ -24,7 +24,8 @@ int main(int argc, char** argv) {
   int code, st = -1;
 
   CHECK(fa_abi_version() == 1);
-  for (code = FA_OK; code <= FA_ERR_TIMEOUT; ++code) CHECK(strcmp(fa_status_string(code), "unknown status") != 0);
+  CHECK(fa_build_flags() == 0 || fa_build_flags() == FA_BUILD_DEBUG);
+  for (code = FA_OK; code <= FA_ERR_BOUNDS; ++code) CHECK(strcmp(fa_status_string(code), "unknown status") != 0);
   CHECK(strcmp(fa_status_string(FA_OK), fa_status_string(FA_ERR_NULL)) != 0);
   CHECK(strcmp(fa_status_string(-1), "unknown status") == 0);
 

@@ -53,12 +53,22 @@ def test_binding_names_match_c_names():
 def test_abi_version_and_status_strings(lib):
     assert fa.fa_abi_version() == 1
     seen = set()
-    for code in range(11):
+    for code in range(12):
         s = fa.fa_status_string(code)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 11
+    assert len(seen) == 12
     assert fa.fa_status_string(999) == "unknown status"
+    assert fa.fa_build_flags() == 0  # the release library
+
+
+def test_debug_library_builds_and_exports_the_same_boundary():
+    from exact_tiled_attention_47_b200 import build
+    path = build.build(debug=True)
+    dbg = fa._lib.load(path)
+    assert dbg.fa_build_flags() == fa.FA_BUILD_DEBUG
+    for n in _declared_functions():
+        assert hasattr(dbg, n), n
 
 
 def test_workspace_bytes(lib):
