@@ -19,7 +19,7 @@ FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 FA_BUILD_DEBUG = 1
 
 __all__ = [
-    "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
+    "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_masked", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_build_flags", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "decode_sharded", "shard_range", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "DEBUG_LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32", "FA_BUILD_DEBUG",
@@ -97,6 +97,22 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, wo
     return lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                       int(B), int(H), int(Nq), int(Nk), int(D), float(scale), int(bool(causal)), _ptr(workspace),
                       int(workspace_bytes), _stream(stream), int(in_dtype), int(grad_dtype))
+
+
+def fa_bwd_masked(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, prefix_len, cu_seqlens,
+                  workspace, workspace_bytes=None, stream=None, in_dtype=None, grad_dtype=None) -> int:
+    """Marshal to the C ``fa_bwd_masked`` (prefix mask, packed varlen); returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if grad_dtype is None:
+        grad_dtype = _dtype_code(dq)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                             _ptr(dv), int(B), int(H), int(Nq), int(Nk), int(D), float(scale), int(bool(causal)),
+                             int(prefix_len), _ptr(cu_seqlens), _ptr(workspace), int(workspace_bytes),
+                             _stream(stream), int(in_dtype), int(grad_dtype))
 
 
 def fa_decode_workspace_bytes(B, H, D, num_splits) -> int:
@@ -249,21 +265,38 @@ def attention(q, k, v, causal=False, scale=None, cu_seqlens=None, out_dtype=None
     return o, lse
 
 
-def attention_backward(q, k, v, o, lse, dout, causal=False, scale=None, grad_dtype=None, stream=None):
-    """dQ, dK, dV for dense q [B,Nq,H,D], k/v [B,Nk,H,D], the forward o / lse and the upstream dout."""
+def attention_backward(q, k, v, o, lse, dout, causal=False, scale=None, grad_dtype=None, stream=None,
+                       prefix_len=None, cu_seqlens=None):
+    """dQ, dK, dV for the forward o / lse and the upstream dout.
+
+    Dense q [B,Nq,H,D], k/v [B,Nk,H,D], or packed [total,H,D] with ``cu_seqlens``; ``prefix_len``
+    (not None) selects the prefix mask of ``attention(..., prefix_len=...)``.
+    """
     import torch
-    B, Nq, H, D = q.shape
-    Nk = k.shape[1]
+    D = q.shape[-1]
+    if cu_seqlens is None:
+        B, Nq, H, _ = q.shape
+        Nk = k.shape[1]
+        nb = fa_bwd_workspace_bytes(B, H, Nq)
+    else:
+        Nq, H, _ = q.shape
+        Nk = k.shape[0]
+        B = cu_seqlens.numel() - 1
+        nb = fa_bwd_workspace_bytes(1, H, Nq)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     grad_dtype = q.dtype if grad_dtype is None else grad_dtype
     dq = torch.empty(q.shape, device=q.device, dtype=grad_dtype)
     dk = torch.empty(k.shape, device=q.device, dtype=grad_dtype)
     dv = torch.empty(v.shape, device=q.device, dtype=grad_dtype)
-    ws = torch.empty(fa_bwd_workspace_bytes(B, H, Nq), device=q.device, dtype=torch.uint8)
-    st = fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, ws, stream=stream)
+    ws = torch.empty(nb, device=q.device, dtype=torch.uint8)
+    if prefix_len is None and cu_seqlens is None:
+        st = fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, ws, stream=stream)
+    else:
+        st = fa_bwd_masked(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal,
+                           0 if prefix_len is None else prefix_len, cu_seqlens, ws, stream=stream)
     if st != FA_OK:
-        raise FAError(st, "fa_bwd")
+        raise FAError(st, "fa_bwd" if prefix_len is None and cu_seqlens is None else "fa_bwd_masked")
     return dq, dk, dv
 
 

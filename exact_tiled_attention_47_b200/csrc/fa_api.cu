@@ -388,23 +388,34 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq) {
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
-           void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal, void* workspace,
-           size_t workspace_bytes, fa_stream_t stream, int in_dtype, int grad_dtype) {
+int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal,
+                  int prefix_len, const int* cu_seqlens, void* workspace, size_t workspace_bytes, fa_stream_t stream,
+                  int in_dtype, int grad_dtype) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
   if (in_dtype != FA_BF16 && in_dtype != FA_FP16) return FA_ERR_DTYPE;
   if (grad_dtype != in_dtype && grad_dtype != FA_FP32) return FA_ERR_DTYPE;
   if (D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || B > 65535 || H > 65535) return FA_ERR_SHAPE;
-  if (Nq > (1 << 24) || Nk > (1 << 24)) return FA_ERR_SHAPE;
-  if (static_cast<int64_t>(B) * Nq >= INT32_MAX || static_cast<int64_t>(B) * Nk >= INT32_MAX) return FA_ERR_SHAPE;
-  if (static_cast<int64_t>(B) * H * ((std::max(Nq, Nk) + 127) / 128) >= INT32_MAX) return FA_ERR_SHAPE;
+  if (prefix_len < 0) return FA_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (cu_seqlens) {
+    if (Nq != Nk) return FA_ERR_SHAPE;  // self-attention: one packed extent for Q and K/V
+    if (static_cast<int64_t>(Nq) / 128 + B > INT32_MAX / 2) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(H) * (Nq / 128 + B) >= INT32_MAX) return FA_ERR_SHAPE;
+  } else {
+    if (Nq > (1 << 24) || Nk > (1 << 24)) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(B) * Nq >= INT32_MAX || static_cast<int64_t>(B) * Nk >= INT32_MAX) return FA_ERR_SHAPE;
+    if (static_cast<int64_t>(B) * H * ((std::max(Nq, Nk) + 127) / 128) >= INT32_MAX) return FA_ERR_SHAPE;
+  }
   if (!fa::aligned(q, 16) || !fa::aligned(k, 16) || !fa::aligned(v, 16) || !fa::aligned(o, 16) ||
       !fa::aligned(dout, 16) || !fa::aligned(dq, 16) || !fa::aligned(dk, 16) || !fa::aligned(dv, 16) ||
       !fa::aligned(lse, 4))
     return FA_ERR_ALIGN;
-  if (!workspace || workspace_bytes < fa_bwd_workspace_bytes(B, H, Nq)) return FA_ERR_WORKSPACE;
+  if (cu_seqlens && !fa::aligned(cu_seqlens, 4)) return FA_ERR_ALIGN;
+  // Drow: one float per query row, [B, H, Nq] dense or [H, total] varlen
+  const size_t ws_need = cu_seqlens ? fa_bwd_workspace_bytes(1, H, Nq) : fa_bwd_workspace_bytes(B, H, Nq);
+  if (!workspace || workspace_bytes < ws_need) return FA_ERR_WORKSPACE;
   if (!fa::aligned(workspace, 16)) return FA_ERR_ALIGN;
   int dev = -1;
   if (const int st = fa::check_device(&dev)) return st;
@@ -422,13 +433,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   a.dv = dv;
   a.drow = static_cast<float*>(workspace);
   a.status = status;
+  a.cu_seqlens = cu_seqlens;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
   a.Nk = Nk;
   a.D = D;
   a.scale = scale;
-  a.causal = causal != 0;
+  a.causal = (causal != 0 || prefix_len > 0) ? 1 : 0;
+  a.prefix = prefix_len;
   a.fp16 = in_dtype == FA_FP16;
   a.g_fp32 = grad_dtype == FA_FP32;
   const int e = fa::launch_backward(a, reinterpret_cast<cudaStream_t>(stream));
@@ -437,6 +450,13 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal, void* workspace,
+           size_t workspace_bytes, fa_stream_t stream, int in_dtype, int grad_dtype) {
+  return fa_bwd_masked(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, D, scale, causal, 0, nullptr, workspace,
+                       workspace_bytes, stream, in_dtype, grad_dtype);
 }
 
 }  // extern "C"

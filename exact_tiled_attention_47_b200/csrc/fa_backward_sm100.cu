@@ -29,7 +29,9 @@
 // P/dS columns).  The MMA forms are those of the forward kernel: SS with both operands K-major (S, dP)
 // and TS with the A operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal runs skip
 // fully masked blocks; masking is applied on the blocks that cross the diagonal and at the sequence
-// ends.
+// ends.  The masks and layouts are those of the forward kernel: causal (bottom-right aligned), the
+// prefix-LM mask (keys [0, prefix) visible to every query of the sequence) and packed varlen
+// sequences indexed through cu_seqlens (LSE and Drow [H, total]).
 #include <cudaTypedefs.h>
 
 #include "fa_prefill_common.cuh"
@@ -65,11 +67,63 @@ struct BwdParams {
   void* g1;           // dv (dkdv kernel)
   long long g0_n, g1_n;  // elements of g0 and g1 (bounds of the debug index checks)
   int* status;
-  int B, H, Nq, Nk;
-  int num_tiles;  // query tiles (dq) or key tiles (dkdv) per (b, h)
+  const int* cu;  // packed varlen: int32[B + 1] sequence starts (nullptr: dense [B, N, H, D])
+  int B, H, Nq, Nk;  // varlen: Nq = Nk = total packed rows
+  int num_tiles;  // dense: query tiles (dq) or key tiles (dkdv) per (b, h); varlen: slots per head
   float scale, scale_log2;
   int causal;
+  int prefix;  // causal only: keys [0, prefix) of a sequence are visible to all of its queries
 };
+
+// The CTA's (batch item, head, 128-row tile) and its sequence: rows [row0, row0 + L) of the packed
+// query / key tensors; head-major order.  Dense: tiles of one (b, h) are consecutive, the tile with
+// the most causal work first (dq: the last query tile; dk/dv: the first key tile).  Varlen: slots of
+// one head are consecutive, sequences in order, tiles found by a warp-wide scan of cu_seqlens; spare
+// slots get b = -1.
+struct BwdUnit {
+  int b, h, tile;
+  int q_row0, k_row0, Lq, Lk;
+};
+
+template <bool kLastFirst>
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, int warp, int lane, int* sh_b, int* sh_t) {
+  BwdUnit u;
+  if (p.cu == nullptr) {
+    const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
+    const int t = static_cast<int>(blockIdx.x % p.num_tiles);
+    u.tile = kLastFirst ? p.num_tiles - 1 - t : t;
+    u.b = bh / p.H;
+    u.h = bh % p.H;
+    u.q_row0 = u.b * p.Nq;
+    u.k_row0 = u.b * p.Nk;
+    u.Lq = p.Nq;
+    u.Lk = p.Nk;
+    return u;
+  }
+  u.h = static_cast<int>(blockIdx.x / p.num_tiles);
+  const int slot = static_cast<int>(blockIdx.x % p.num_tiles);
+  if (warp == 0) {
+    FwdParams f{};  // the unit finder reads cu, B, Nq and status
+    f.cu = p.cu;
+    f.B = p.B;
+    f.Nq = p.Nq;
+    f.status = p.status;
+    int fb, fm;
+    find_varlen_unit<kBT>(f, slot, lane, fb, fm);  // fm counts the sequence's tiles from its last
+    if (lane == 0) {
+      *sh_b = fb;
+      *sh_t = fm;
+    }
+  }
+  __syncthreads();
+  u.b = *sh_b;
+  u.tile = *sh_t;
+  if (u.b < 0) return u;
+  u.q_row0 = u.k_row0 = p.cu[u.b];
+  u.Lq = u.Lk = p.cu[u.b + 1] - p.cu[u.b];
+  if (!kLastFirst) u.tile = (u.Lq + kBT - 1) / kBT - 1 - u.tile;
+  return u;
+}
 
 struct BwdBars {
   uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
@@ -79,6 +133,7 @@ struct BwdBars {
   uint64_t o_done, drain;
   uint32_t tmem_base;
   int abort_flag;
+  int unit_b, unit_t;
 };
 static_assert(sizeof(BwdBars) <= 256, "barrier block too large");
 
@@ -256,19 +311,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
-  const int m_block = p.num_tiles - 1 - static_cast<int>(blockIdx.x % p.num_tiles);  // longest first
-  const int b = bh / p.H, h = bh % p.H;
-  const int m0 = m_block * kBT;
-  const int Lq = p.Nq, Lk = p.Nk, diag = Lk - Lq;
+  const BwdUnit u = bwd_unit<true>(p, warp, lane, &bars->unit_b, &bars->unit_t);
+  if (u.b < 0) return;  // spare varlen slot (uniform across the CTA)
+  const int b = u.b, h = u.h;
+  const int m0 = u.tile * kBT;
+  const int Lq = u.Lq, Lk = u.Lk, diag = Lk - Lq;
   int kv_end = Lk;
-  if (p.causal) kv_end = min(Lk, m0 + kBT + diag);
-  const int n = (kv_end > 0) ? (kv_end + kBT - 1) / kBT : 0;
+#ifndef FA_DEBUG
+  if (p.causal) kv_end = min(Lk, max(p.prefix, m0 + kBT + diag));
+#endif
+  const int n = (m0 < Lq && kv_end > 0) ? (kv_end + kBT - 1) / kBT : 0;
   if (n == 0) {  // no row of the tile sees a key: dQ = 0
     if (warp < 4) {
       const int qi = m0 + warp * 32 + lane;
       if (qi < Lq) {
-        const size_t row = ((static_cast<size_t>(b) * Lq + qi) * p.H + h) * D;
+        const size_t row = (static_cast<size_t>(u.q_row0 + qi) * p.H + h) * D;
         for (int d = 0; d < D && idx_ok(p.status, row, D, p.g0_n); ++d) {
           if constexpr (kOutF32) static_cast<float*>(p.g0)[row + d] = 0.f;
           else static_cast<uint16_t*>(p.g0)[row + d] = 0;
@@ -287,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::kTileBytes);
 #pragma unroll
       for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_3d(&tm_q, &bars->fixed_full, sQ + pn * kPanelBytes, pn * 64, h, b * Lq + m0);
-        tma_load_3d(&tm_do, &bars->fixed_full, sDO + pn * kPanelBytes, pn * 64, h, b * Lq + m0);
+        tma_load_3d(&tm_q, &bars->fixed_full, sQ + pn * kPanelBytes, pn * 64, h, u.q_row0 + m0);
+        tma_load_3d(&tm_do, &bars->fixed_full, sDO + pn * kPanelBytes, pn * 64, h, u.q_row0 + m0);
       }
       int issued = 0;
       bool ok = true;
@@ -298,8 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d_hint(&tm_k, &bars->st_full[st], sK(st) + pn * kPanelBytes, pn * 64, h, b * Lk + j * kBT, keep);
-          tma_load_3d_hint(&tm_v, &bars->st_full[st], sV(st) + pn * kPanelBytes, pn * 64, h, b * Lk + j * kBT, keep);
+          tma_load_3d_hint(&tm_k, &bars->st_full[st], sK(st) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
+          tma_load_3d_hint(&tm_v, &bars->st_full[st], sV(st) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
         }
         issued = j + 1;
       }
@@ -353,10 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;
     const int qi = m0 + r;
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int row_lim = p.causal ? min(Lk, qi + 1 + diag) : Lk;
-    const int tile_lim = p.causal ? min(Lk, m0 + 1 + diag) : Lk;
-    const size_t stat = (static_cast<size_t>(b) * p.H + h) * Lq + min(qi, Lq - 1);
-    const bool stat_in = idx_ok(p.status, stat, 1, static_cast<long long>(p.B) * p.H * Lq);
+    // keys [0, row_lim) are visible to this row; tile_lim is the smallest row_lim of the tile
+    const int row_lim = p.causal ? min(Lk, max(p.prefix, qi + 1 + diag)) : Lk;
+    const int tile_lim = p.causal ? min(Lk, max(p.prefix, m0 + 1 + diag)) : Lk;
+    // LSE and Drow: [B, H, Nq] dense, [H, total] varlen
+    const size_t stat = (p.cu == nullptr ? (static_cast<size_t>(b) * p.H + h) * p.Nq
+                                         : static_cast<size_t>(h) * p.Nq + u.q_row0) + min(qi, Lq - 1);
+    const bool stat_in = idx_ok(p.status, stat, 1, static_cast<long long>(p.cu == nullptr ? p.B : 1) * p.H * p.Nq);
     const float lse = stat_in ? p.lse[stat] : -INFINITY;
     // rows without keys (LSE = -inf) and rows past the end get P = 0
     const float lse2 = (qi < Lq && lse != -INFINITY) ? lse * kLog2e : INFINITY;
@@ -404,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
-      const size_t row = (static_cast<size_t>(b) * Lq + min(qi, Lq - 1)) * p.H + h;
+      const size_t row = static_cast<size_t>(u.q_row0 + min(qi, Lq - 1)) * p.H + h;
       // the two halves of warps store the two halves of the row
       store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, p.status, p.g0_n,
                                         hh * D / 64, (hh + 1) * D / 64);
@@ -433,20 +493,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
-  const int n_block = static_cast<int>(blockIdx.x % p.num_tiles);  // causal: the first key tile sees most
-  const int b = bh / p.H, h = bh % p.H;
-  const int n0 = n_block * kBT;
-  const int Lq = p.Nq, Lk = p.Nk, diag = Lk - Lq;
-  // query blocks that see any key of this tile: q >= k - diag for the tile's first key k = n0
-  const int i_first = p.causal ? max(0, n0 - diag) / kBT : 0;
+  const BwdUnit u = bwd_unit<false>(p, warp, lane, &bars->unit_b, &bars->unit_t);
+  if (u.b < 0) return;  // spare varlen slot (uniform across the CTA)
+  const int b = u.b, h = u.h;
+  const int n0 = u.tile * kBT;
+  const int Lq = u.Lq, Lk = u.Lk, diag = Lk - Lq;
+  // query blocks that see any key of this tile: every query if the tile starts inside the prefix,
+  // else q >= k - diag for the tile's first key k = n0 (causal)
+  bool skip = p.causal && n0 >= p.prefix;
+#ifdef FA_DEBUG
+  skip = false;  // the debug build walks every query block and lets the mask zero the invisible ones
+#endif
+  const int i_first = skip ? max(0, n0 - diag) / kBT : 0;
   const int nq_blocks = (Lq + kBT - 1) / kBT;
-  const int n = (p.causal && n0 - diag > Lq - 1) ? 0 : nq_blocks - i_first;
+  const int n = (n0 >= Lk || (skip && n0 - diag > Lq - 1)) ? 0 : nq_blocks - i_first;
   if (n <= 0) {  // no query sees this tile: dK = dV = 0
     if (warp < 4) {
       const int kj = n0 + warp * 32 + lane;
       if (kj < Lk) {
-        const size_t row = ((static_cast<size_t>(b) * Lk + kj) * p.H + h) * D;
+        const size_t row = (static_cast<size_t>(u.k_row0 + kj) * p.H + h) * D;
         for (int d = 0; d < D && idx_ok(p.status, row, D, p.g0_n) && idx_ok(p.status, row, D, p.g1_n); ++d) {
           if constexpr (kOutF32) {
             static_cast<float*>(p.g0)[row + d] = 0.f;
@@ -470,8 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::kTileBytes);
 #pragma unroll
       for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_3d(&tm_k, &bars->fixed_full, sK + pn * kPanelBytes, pn * 64, h, b * Lk + n0);
-        tma_load_3d(&tm_v, &bars->fixed_full, sV + pn * kPanelBytes, pn * 64, h, b * Lk + n0);
+        tma_load_3d(&tm_k, &bars->fixed_full, sK + pn * kPanelBytes, pn * 64, h, u.k_row0 + n0);
+        tma_load_3d(&tm_v, &bars->fixed_full, sV + pn * kPanelBytes, pn * 64, h, u.k_row0 + n0);
       }
     }
     int issued = 0;
@@ -483,27 +548,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d_hint(&tm_q, &bars->st_full[st], sQ(st) + pn * kPanelBytes, pn * 64, h, b * Lq + i * kBT, keep);
-          tma_load_3d_hint(&tm_do, &bars->st_full[st], sDO(st) + pn * kPanelBytes, pn * 64, h, b * Lq + i * kBT, keep);
+          tma_load_3d_hint(&tm_q, &bars->st_full[st], sQ(st) + pn * kPanelBytes, pn * 64, h, u.q_row0 + i * kBT, keep);
+          tma_load_3d_hint(&tm_do, &bars->st_full[st], sDO(st) + pn * kPanelBytes, pn * 64, h, u.q_row0 + i * kBT, keep);
         }
       }
       issued = jj + 1;
       // the block's LSE (log2 units; +inf for rows without keys or past the end, so P = 0) and Drow:
       // all eight loads of a lane are independent and in flight together
       float* stat = sStat + st * 2 * kBT;
-      const size_t base = (static_cast<size_t>(b) * p.H + h) * Lq;
+      // LSE and Drow: [B, H, Nq] dense, [H, total] varlen
+      const size_t base = p.cu == nullptr ? (static_cast<size_t>(b) * p.H + h) * p.Nq
+                                          : static_cast<size_t>(h) * p.Nq + u.q_row0;
+      const long long stat_n = static_cast<long long>(p.cu == nullptr ? p.B : 1) * p.H * p.Nq;
       float lv[4], dv[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int qi = i * kBT + lane + 32 * u;
-        const bool in = qi < Lq && idx_ok(p.status, base + qi, 1, static_cast<long long>(p.B) * p.H * Lq);
-        lv[u] = in ? p.lse[base + qi] : -INFINITY;
-        dv[u] = in ? p.drow[base + qi] : 0.f;
+      for (int e = 0; e < 4; ++e) {
+        const int qi = i * kBT + lane + 32 * e;
+        const bool in = qi < Lq && idx_ok(p.status, base + qi, 1, stat_n);
+        lv[e] = in ? p.lse[base + qi] : -INFINITY;
+        dv[e] = in ? p.drow[base + qi] : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        stat[lane + 32 * u] = (lv[u] != -INFINITY) ? lv[u] * kLog2e : INFINITY;
-        stat[kBT + lane + 32 * u] = dv[u];
+      for (int e = 0; e < 4; ++e) {
+        stat[lane + 32 * e] = (lv[e] != -INFINITY) ? lv[e] * kLog2e : INFINITY;
+        stat[kBT + lane + 32 * e] = dv[e];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->stat_full[st]);  // release: orders the warp's stores above
@@ -568,10 +636,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(&bars->stat_full[st], (jj / C::kSt) & 1, abort_flag, p.status))) break;
       tc_fence_after();
       const float* stat = sStat + st * 2 * kBT;
-      // key kj is visible to query q iff q >= kj - diag (causal); whole block visible iff its first
-      // query already sees the tile's last key
+      // key kj is visible to query q iff kj < prefix or q >= kj - diag (causal); the whole block is
+      // visible iff its first query already sees the tile's last key; queries past the sequence end
+      // have P = 0 through their +inf LSE
       const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
-      const int q_lo = kj - diag - i * kBT;  // columns c < q_lo are masked
+      const int q_lo = (kj < p.prefix) ? -kBT : kj - diag - i * kBT;  // columns c < q_lo are masked
       // the half's 64 query columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
       const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
       uint32_t sb[2][16], db[2][16];
@@ -617,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
-      const size_t row = ((static_cast<size_t>(b) * Lk + min(kj, Lk - 1)) * p.H + h) * D;
+      const size_t row = (static_cast<size_t>(u.k_row0 + min(kj, Lk - 1)) * p.H + h) * D;
       if (hh == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk, p.status, p.g1_n);  // dV
       else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk, p.status, p.g0_n);  // dK
     }
@@ -628,9 +697,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, bool kFp16, bool kOutF32>
 int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, cudaStream_t stream) {
   const int smem = BwdCfg<D>::kSmemBytes;
-  const size_t rows = static_cast<size_t>(a.B) * a.Nq * a.H;
-  bwd_rowterm_kernel<kFp16, D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(a.o, a.dout, a.drow,
-                                                                                             a.B, a.H, a.Nq, a.status);
+  const bool varlen = a.cu_seqlens != nullptr;
+  const size_t rows = static_cast<size_t>(varlen ? 1 : a.B) * a.Nq * a.H;
+  // varlen rows are those of one batch item of Nq = total rows: Drow [H, total]
+  bwd_rowterm_kernel<kFp16, D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
+      a.o, a.dout, a.drow, varlen ? 1 : a.B, a.H, a.Nq, a.status);
   auto kq = bwd_dq_kernel<D, kFp16, kOutF32>;
   auto kkv = bwd_dkdv_kernel<D, kFp16, kOutF32>;
   // the shared-memory opt-in is a per-device (per-context) attribute: raised once
@@ -644,15 +715,17 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   if (ce != 0) return ce;
   BwdParams pq = p;
   pq.g0 = a.dq;
-  pq.g0_n = static_cast<long long>(a.B) * a.Nq * a.H * D;
-  pq.num_tiles = (a.Nq + kBT - 1) / kBT;
-  kq<<<static_cast<unsigned>(pq.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pq);
+  pq.g0_n = static_cast<long long>(varlen ? 1 : a.B) * a.Nq * a.H * D;
+  // dense: tiles per (b, h); varlen: slots per head, enough for the sum over the sequences of
+  // ceil(len / 128) <= total / 128 + B (spare slots exit at once)
+  pq.num_tiles = varlen ? a.Nq / kBT + a.B : (a.Nq + kBT - 1) / kBT;
+  kq<<<static_cast<unsigned>(pq.num_tiles * (varlen ? 1 : a.B) * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pq);
   BwdParams pk = p;
   pk.g0 = a.dk;
   pk.g1 = a.dv;
-  pk.g0_n = pk.g1_n = static_cast<long long>(a.B) * a.Nk * a.H * D;
-  pk.num_tiles = (a.Nk + kBT - 1) / kBT;
-  kkv<<<static_cast<unsigned>(pk.num_tiles * a.B * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pk);
+  pk.g0_n = pk.g1_n = static_cast<long long>(varlen ? 1 : a.B) * a.Nk * a.H * D;
+  pk.num_tiles = varlen ? a.Nk / kBT + a.B : (a.Nk + kBT - 1) / kBT;
+  kkv<<<static_cast<unsigned>(pk.num_tiles * (varlen ? 1 : a.B) * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pk);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -660,10 +733,12 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
 
 int launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   CUtensorMap m[4];
-  if (!make_tma_map(&m[0], a.q, a.B * a.Nq, a.H, a.D, a.fp16, kBT) ||
-      !make_tma_map(&m[1], a.dout, a.B * a.Nq, a.H, a.D, a.fp16, kBT) ||
-      !make_tma_map(&m[2], a.k, a.B * a.Nk, a.H, a.D, a.fp16, kBT) ||
-      !make_tma_map(&m[3], a.v, a.B * a.Nk, a.H, a.D, a.fp16, kBT))
+  const int rows_q = a.cu_seqlens != nullptr ? a.Nq : a.B * a.Nq;
+  const int rows_k = a.cu_seqlens != nullptr ? a.Nk : a.B * a.Nk;
+  if (!make_tma_map(&m[0], a.q, rows_q, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[1], a.dout, rows_q, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[2], a.k, rows_k, a.H, a.D, a.fp16, kBT) ||
+      !make_tma_map(&m[3], a.v, rows_k, a.H, a.D, a.fp16, kBT))
     return static_cast<int>(cudaErrorInvalidValue);
   BwdParams p;
   p.lse = a.lse;
@@ -679,6 +754,8 @@ int launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal ? 1 : 0;
+  p.prefix = a.causal ? a.prefix : 0;
+  p.cu = a.cu_seqlens;
   if (a.D == 64) {
     if (a.fp16) return a.g_fp32 ? launch_bwd_t<64, true, true>(a, m, p, stream) : launch_bwd_t<64, true, false>(a, m, p, stream);
     return a.g_fp32 ? launch_bwd_t<64, false, true>(a, m, p, stream) : launch_bwd_t<64, false, false>(a, m, p, stream);

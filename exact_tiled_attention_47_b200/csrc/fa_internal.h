@@ -69,11 +69,13 @@ struct BackwardArgs {
   void* dq;
   void* dk;
   void* dv;
-  float* drow;  // workspace: [B, H, Nq] fp32
+  float* drow;  // workspace: [B, H, Nq] fp32 ([H, total] varlen)
   int* status;
+  const int* cu_seqlens = nullptr;  // packed varlen (Nq = Nk = total); nullptr = dense
   int B, H, Nq, Nk, D;
   float scale;
   int causal;
+  int prefix = 0;  // causal only: keys [0, prefix) are visible to every query
   int fp16;    // input type: 1 = fp16, 0 = bf16
   int g_fp32;  // gradient type: 1 = fp32, 0 = input type
 };

@@ -128,13 +128,36 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq);
  * fp32 as written by fa_fwd with the same q, k, v, scale and causal; dq [B, Nq, H, D] and dk, dv
  * [B, Nk, H, D] of grad_dtype (in_dtype or FA_FP32), fully overwritten.  causal as fa_fwd
  * (bottom-right aligned).  workspace: device buffer of at least fa_bwd_workspace_bytes(B, H, Nq)
- * bytes, owned by the caller, 16-byte aligned.  No varlen or prefix form.  Limits and errors as
- * fa_fwd (FA_ERR_WORKSPACE for a missing or short workspace).  A query row with LSE = -inf (no
- * visible key) contributes nothing.  Three kernels run in order on `stream`; nothing is allocated.
+ * bytes, owned by the caller, 16-byte aligned.  The prefix-mask and varlen forms are
+ * fa_bwd_masked.  Limits and errors as fa_fwd (FA_ERR_WORKSPACE for a missing or short workspace).
+ * A query row with LSE = -inf (no visible key) contributes nothing.  Three kernels run in order on
+ * `stream`; nothing is allocated.  Same as fa_bwd_masked with prefix_len = 0, cu_seqlens = NULL.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal,
            void* workspace, size_t workspace_bytes, fa_stream_t stream, int in_dtype, int grad_dtype);
+
+/*
+ * fa_bwd_masked -- gradients of every forward form: the backward of fa_fwd (dense or packed
+ * varlen, causal or not) and of fa_fwd_prefix.
+ *
+ * Passages: those of fa_bwd for the gradients; the masks are the forward's (causal, bottom-right
+ * aligned; the prefix-LM mask of fa_fwd_prefix, where prefix_len > 0 makes the first prefix_len keys
+ * of each sequence visible to all its queries and implies causal); the varlen layout is that of
+ * fa_fwd with cu_seqlens (Hugging Face page, FAQ 4 and "常见错误排查", error 4).
+ *
+ * Dense (cu_seqlens == NULL): layouts and lse as fa_bwd.  Varlen (cu_seqlens != NULL, int32[B + 1]
+ * on the device, as given to fa_fwd): q, k, v, o, dout, dq, dk, dv are packed [total, H, D] with
+ * Nq = Nk = total, lse is [H, total] as fa_fwd wrote it, and the workspace needs
+ * fa_bwd_workspace_bytes(1, H, total) bytes.  lse must come from the forward call with the same
+ * inputs, scale and mask.  Errors as fa_bwd, plus FA_ERR_SHAPE for prefix_len < 0 or Nq != Nk with
+ * cu_seqlens, FA_ERR_ALIGN for a misaligned cu_seqlens; an inconsistent cu_seqlens is reported on
+ * the device as FA_ERR_CU_SEQLENS (fa_device_status) and its tiles are skipped.
+ */
+int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D, float scale, int causal,
+                  int prefix_len, const int* cu_seqlens, void* workspace, size_t workspace_bytes,
+                  fa_stream_t stream, int in_dtype, int grad_dtype);
 
 /*
  * fa_decode_workspace_bytes -- size of the scratch buffer fa_decode_splitkv needs:

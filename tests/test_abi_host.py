@@ -223,6 +223,28 @@ def test_bwd_validation_codes(lib):
     assert fa.fa_bwd_workspace_bytes(2, 3, 100) == 2560  # 2*3*100*4 = 2400 rounded up to 256
 
 
+def test_bwd_masked_validation_codes(lib):
+    def bwd(**kw):
+        a = dict(q=A, k=A, v=A, o=A, do=A, lse=A, dq=A, dk=A, dv=A, B=2, H=3, Nq=300, Nk=300, D=64, scale=0.125,
+                 causal=1, prefix=0, cu=None, ws=A, wsb=1 << 20, in_dtype=0, g_dtype=0)
+        a.update(kw)
+        return lib.fa_bwd_masked(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                                 a["B"], a["H"], a["Nq"], a["Nk"], a["D"], a["scale"], a["causal"], a["prefix"],
+                                 a["cu"], a["ws"], a["wsb"], None, a["in_dtype"], a["g_dtype"])
+    assert bwd(lse=None) == fa.FA_ERR_NULL
+    assert bwd(g_dtype=1) == fa.FA_ERR_DTYPE
+    assert bwd(D=80) == fa.FA_ERR_HEADDIM
+    assert bwd(prefix=-1) == fa.FA_ERR_SHAPE
+    assert bwd(cu=A, Nk=299) == fa.FA_ERR_SHAPE          # varlen is self-attention: Nq == Nk
+    assert bwd(cu=A + 2) == fa.FA_ERR_ALIGN
+    assert bwd(q=A + 4) == fa.FA_ERR_ALIGN
+    # varlen needs one row term per packed row and head: H * total floats, whatever B is
+    need = fa.fa_bwd_workspace_bytes(1, 3, 300)
+    assert bwd(cu=A, wsb=need - 1) == fa.FA_ERR_WORKSPACE
+    assert bwd(cu=A, ws=None) == fa.FA_ERR_WORKSPACE
+    assert bwd(wsb=fa.fa_bwd_workspace_bytes(2, 3, 300) - 1) == fa.FA_ERR_WORKSPACE
+
+
 def test_device_status_null(lib):
     assert lib.fa_device_status(None, 0) == fa.FA_ERR_NULL
 
@@ -236,6 +258,8 @@ def test_no_device_is_reported(lib):
     w = ctypes.c_int(0)
     assert lib.fa_selftest_wait_timeout(ctypes.byref(w), None) == fa.FA_ERR_DEVICE
     assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, 128, 64, 0.125, 0, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
+    assert lib.fa_bwd_masked(A, A, A, A, A, A, A, A, A, 2, 1, 300, 300, 64, 0.125, 1, 7, A, A, 1 << 20, None, 0,
+                             0) == fa.FA_ERR_DEVICE
     assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
     assert _shard(lib) == fa.FA_ERR_DEVICE
     assert _shard(lib, off=64, sl=A) == fa.FA_ERR_DEVICE

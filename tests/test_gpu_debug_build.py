@@ -6,10 +6,10 @@ and, instead of touching memory outside it, records FA_ERR_BOUNDS in the device 
 tests run every entry point of the debug library on ragged and edge shapes and require the status
 word to stay clear and the results to match the fp64 oracle.
 
-The same build also turns off the causal block skip of the prefill kernel: it walks every key block
-of a tile and lets the mask zero the invisible ones.  Skipping a fully masked block must change
-nothing -- its P is exactly zero -- so the release library's output must equal the debug library's
-bit for bit (causal, with Nq < Nk and Nq > Nk, the prefix mask, packed varlen).
+The same build also turns off the causal block skip of the prefill and backward kernels: they walk
+every key (query) block and let the mask zero the invisible ones.  Skipping a fully masked block must
+change nothing -- its P is exactly zero -- so the release library's outputs and gradients must equal
+the debug library's bit for bit (causal, with Nq < Nk and Nq > Nk, the prefix mask, packed varlen).
 """
 import math
 
@@ -186,3 +186,38 @@ def test_debug_noalloc_decode(use_debug):
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attention_decode(to_f64(q, "bf16"), to_f64(k, "bf16"), to_f64(v, "bf16"), 1 / math.sqrt(D))
     check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref[:, :, 0], "fp32", "debug noalloc")
+
+
+@pytest.mark.parametrize("prefix,cu", [(0, False), (90, False), (0, True)])
+def test_backward_skip_equals_mask_everything(libs, monkeypatch, prefix, cu):
+    """The backward's causal block skip (dQ: key blocks past the diagonal; dK/dV: query blocks before
+    it) changes nothing: the release library's gradients equal the debug library's bit for bit."""
+    fa, rel, dbg = libs
+    scale = 0.125
+    if cu:
+        q, k, v, cus = si.varlen_qkv(8900, [300, 1, 129, 0, 260], 2, 64, "bf16")
+        total = int(cus[-1])
+        do = si.batch_item(8900, 3, 0, (total, 2, 64), "bf16")
+        kw = dict(cu_seqlens=torch.from_numpy(cus).cuda())
+    else:
+        q, k, v = si.dense_qkv(8900 + prefix, 2, 333, 333, 2, 64, "bf16")
+        do = si.batched(8900 + prefix, 3, 2, (333, 2, 64), "bf16")
+        kw = {}
+    if prefix:
+        kw["prefix_len"] = prefix
+    args = [to_device(t, "bf16") for t in (q, k, v)]
+    dod = to_device(do, "bf16")
+
+    def run():
+        o, lse = fa.attention(*args, causal=True, scale=scale, **kw)
+        return fa.attention_backward(*args, o, lse, dod, causal=True, scale=scale, grad_dtype=torch.float32, **kw)
+
+    g1 = run()
+    torch.cuda.synchronize()
+    monkeypatch.setattr(fa._lib, "_lib", dbg)
+    fa.fa_device_status(clear=True)
+    g2 = run()
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(clear=True) == 0
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)

@@ -189,3 +189,26 @@ def test_noalloc_decode_writes_stay_inside():
     finish(fa, og, lg)
     o_ref, lse_ref = oracle.attention_decode(to_f64(q, dtype), to_f64(k, dtype), to_f64(v, dtype), scale)
     check(og.t.cpu().numpy(), lg.t.cpu().numpy(), o_ref, lse_ref[:, :, 0], "fp32", "guarded noalloc")
+
+
+def test_masked_backward_writes_stay_inside():
+    fa = fa_mod()
+    lengths, H, D, dtype, prefix = [300, 1, 0, 129], 2, 128, "bf16", 50
+    q, k, v, cu = si.varlen_qkv(7700, lengths, H, D, dtype)
+    total = int(cu[-1])
+    do = si.batch_item(7700, 3, 0, (total, H, D), dtype)
+    qd, kd, vd, dod = (to_device(t, dtype) for t in (q, k, v, do))
+    cut = torch.from_numpy(cu).cuda()
+    o, lse = fa.attention(qd, kd, vd, scale=0.1, cu_seqlens=cut, prefix_len=prefix)
+    gs = [Guarded((total, H, D), torch.float32) for _ in range(3)]
+    nb = fa.fa_bwd_workspace_bytes(1, H, total)
+    wg = Guarded((nb,), torch.uint8)
+    st = fa.fa_bwd_masked(qd, kd, vd, o, dod, lse, gs[0].t, gs[1].t, gs[2].t, len(lengths), H, total, total, D, 0.1,
+                          1, prefix, cut, wg.t, nb)
+    assert st == fa.FA_OK, fa.fa_status_string(st)
+    finish(fa, *gs, wg)
+    refs = oracle.attention_varlen_backward(to_f64(q, dtype), to_f64(k, dtype), to_f64(v, dtype), to_f64(do, dtype),
+                                            cu, 0.1, True, prefix)
+    for name, g, r in zip(("dq", "dk", "dv"), gs, refs):
+        m = max(np.abs(r).max(), 1e-6)
+        assert np.abs(g.t.cpu().numpy() - r).max() / m <= 2e-2, name
