@@ -36,23 +36,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Wait of a whole warp for a barrier phase; true only if the phase completed.
-#ifndef FA_LANE0_WAIT
-#define FA_LANE0_WAIT 0
-#endif
+// Wait by every lane of a warp; true only if all lanes saw the phase complete.  (Polling by one
+// lane with a broadcast was measured slower in the prefill.)
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status) {
-#if FA_LANE0_WAIT
-  // one lane polls the barrier; __syncwarp then orders the other lanes after its acquire
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok;
-#else
   const bool ok = mbar_wait(bar, parity, abort_flag, status);
   return __all_sync(0xffffffffu, ok);
-#endif
 }
 
 // Varlen: map a linear slot to (sequence, unit of kUnitRows query rows) by a warp-wide scan of

@@ -365,14 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         uint32_t sr[128];
         tmem_ld128_sync(lane_base + C::col_s(t), sr);
-#ifndef FA_LATE_SFREE
-#define FA_LATE_SFREE 0
-#endif
-        if (!FA_LATE_SFREE) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may now be overwritten by S_t(j+1)
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may now be overwritten by S_t(j+1)
         const bool masked = (j + 1) * kBN > tile_lim;
         if (masked) {
           const int lim = row_lim - j * kBN;
@@ -381,11 +376,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
         const float m_new = fmaxf(m_run, row_max(sr) * sl2);  // raw score units, scaled
-        if (FA_LATE_SFREE) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may now be overwritten by S_t(j+1)
-        }
         // Rescale O only when the max grew by more than the threshold (warp-uniform decision); the
         // multiplication of O waits below until P_t(j-1) V has landed in O.
         const bool need = m_new > m_run + kRescaleThreshold;
