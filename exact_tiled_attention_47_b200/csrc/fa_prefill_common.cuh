@@ -25,6 +25,8 @@ struct FwdParams {
   float scale_log2;
   int causal;
   int prefix;  // causal only: keys [0, prefix) of a sequence are visible to all its queries
+  int head_group;  // dense: heads whose work units are ordered together, longest first
+  int tma_out;     // 16-bit O: full tiles are written through shared memory by a TMA store
 };
 
 // Bounded wait used only on the abort path: ignores the abort flag, has its own limit.
@@ -194,6 +196,31 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_taddr, 
     }
   }
   if (store) p.lse[lse_index(p, b, h, q_row0, qi)] = empty ? -INFINITY : (m_run + lg2(l_run)) * kLn2;
+}
+
+// Normalises one row of O (O / l, from its fp32 accumulator in TMEM) into a 16-bit tile in shared
+// memory laid out as the TMA tile box reads and writes it: 64-column panels of 128-byte rows, the
+// 16-byte chunks of row r XOR-ed with r mod 8 (128-byte swizzle).
+template <int D, bool kFp16>
+__device__ __forceinline__ void stage_row(uint32_t o_taddr, uint8_t* tile, int r, float m_run, float l_run) {
+  const bool empty = (m_run == -INFINITY);
+  const float inv_l = empty ? 0.f : 1.f / l_run;
+  const uint32_t base = smem_addr(tile) + r * 128;
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t orr[32];
+    tmem_ld32_sync(o_taddr + ch * 32, orr);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float* f = reinterpret_cast<const float*>(orr + 8 * i);
+      const int col = ch * 32 + 8 * i;  // first of 8 output columns = one 16-byte chunk
+      const uint32_t addr = base + (col >> 6) * (128 * 128) + ((((col & 63) >> 3) ^ (r & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                   "r"(pack2<kFp16>(f[0] * inv_l, f[1] * inv_l)), "r"(pack2<kFp16>(f[2] * inv_l, f[3] * inv_l)),
+                   "r"(pack2<kFp16>(f[4] * inv_l, f[5] * inv_l)), "r"(pack2<kFp16>(f[6] * inv_l, f[7] * inv_l))
+                   : "memory");
+    }
+  }
 }
 
 // 3-D TMA map over a [rows, H, D] 16-bit tensor: box = 64 columns x 1 head x box_rows rows, 128-byte

@@ -32,6 +32,7 @@
 // share its K/V in L2.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "fa_prefill_common.cuh"
@@ -115,7 +116,8 @@ __device__ __forceinline__ void store_p_smem(uint32_t tile_base, int r, int ch, 
 template <int D, bool kFp16, bool kOutF32>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
+                  const FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -129,8 +131,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.cu == nullptr) {
     // all pairs of one (b, h) are consecutive, so they run together and share its K/V in L2;
     // within a head the pair with the most key blocks (causal) goes first
-    const int bh = static_cast<int>(blockIdx.x / p.num_units);
-    pair = p.num_units - 1 - static_cast<int>(blockIdx.x % p.num_units);
+    // Groups of head_group (b, h) heads run one after another, so the K/V of the heads in flight
+    // stay in L2; inside a group the pairs with the most key blocks (causal) of all its heads come
+    // first, heads fastest, so that the longest units start early and none is left for the end.
+    const int bhs = p.B * p.H;
+    const int per_group = p.head_group * p.num_units;
+    const int grp = static_cast<int>(blockIdx.x / per_group), w = static_cast<int>(blockIdx.x % per_group);
+    const int gsz = min(p.head_group, bhs - grp * p.head_group);
+    const int bh = grp * p.head_group + w % gsz;
+    pair = p.num_units - 1 - w / gsz;
     b = bh / p.H;
     h = bh % p.H;
   } else {
@@ -442,10 +451,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the last P_t V product (the issuer's MMAs complete in order, so all earlier ones are done)
       if (ok) ok = warp_wait(&bars->o_done[t], (n - 1) & 1, abort_flag, p.status);
-      if (ok) {
+      float l0, l1;
+      f2_split(lsum, l0, l1);
+      if (!kOutF32 && p.tma_out && tile_m0 + kBM <= Lq) {
+        // a full tile of 16-bit O: rows normalised into shared memory (the tile's Q buffer, which no
+        // MMA reads any more), one TMA store per 64-column panel.  All four warps of the tile reach
+        // the named barrier, whether or not their loop completed.
+        if (ok) {
+          tc_fence_after();
+          stage_row<D, kFp16>(lane_base + C::col_o(t), sQ(t), r, m_run, l0 + l1);
+          const size_t li = lse_index(p, b, h, q_row0, qi);
+          if (idx_ok(p.status, li, 1, lse_elems(p))) p.lse[li] = (m_run == -INFINITY) ? -INFINITY : (m_run + lg2(l0 + l1)) * kLn2;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_barrier(1 + t, 128);
+        if (quarter == 0 && lane == 0 && *abort_flag == 0) {
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_store_3d(&tmap_o, sQ(t) + pn * kPanelBytes, pn * 64, h, q_row0 + tile_m0);
+          tma_store_commit();
+          tma_store_wait_read();  // the buffer is released with the CTA
+        }
+      } else if (ok) {
         tc_fence_after();
-        float l0, l1;
-        f2_split(lsum, l0, l1);
         write_row<D, kFp16, kOutF32>(p, lane_base + C::col_o(t), b, h, q_row0, qi, qi < Lq, m_run, l0 + l1);
       }
     }
@@ -462,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool kFp16, bool kOutF32>
 int launch_t(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-             const FwdParams& p, cudaStream_t stream) {
+             const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
   auto kern = fa_fwd_kernel<D, kFp16, kOutF32>;
   const int smem = Cfg<D>::kSmemBytes;
   // Once per device and context: raise the shared-memory limit and confirm the register count the
@@ -484,7 +512,7 @@ int launch_t(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
   else  // sum over sequences of ceil(len / 256) <= total / 256 + B; spare slots exit at once
     blocks = (static_cast<long long>(a.Nq) / (kTiles * kBM) + a.B) * a.H;
   if (blocks > 0x7fffffffLL) return static_cast<int>(cudaErrorInvalidConfiguration);
-  kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(mq, mk, mv, p);
+  kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(mq, mk, mv, mo, p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -521,10 +549,13 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   const bool varlen = a.cu_seqlens != nullptr;
   const int rows_q = varlen ? a.Nq : a.B * a.Nq;
   const int rows_k = varlen ? a.Nk : a.B * a.Nk;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tma_map(&mq, a.q, rows_q, a.H, a.D, a.fp16, kBM) || !make_tma_map(&mk, a.k, rows_k, a.H, a.D, a.fp16, kBN) ||
       !make_tma_map(&mv, a.v, rows_k, a.H, a.D, a.fp16, kBN))
     return static_cast<int>(cudaErrorInvalidValue);
+  // 16-bit O is stored by TMA (same box as Q); an fp32 O keeps the per-thread stores
+  if (a.o_fp32) mo = mq;
+  else if (!make_tma_map(&mo, a.o, rows_q, a.H, a.D, a.fp16, kBM)) return static_cast<int>(cudaErrorInvalidValue);
   FwdParams p;
   p.o = a.o;
   p.lse = a.lse;
@@ -538,12 +569,27 @@ int launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal ? 1 : 0;
   p.prefix = a.causal ? a.prefix : 0;
+  // about FA_GROUP_KV_MB of K and V per head group (half of L2: measured best of 8-64 heads at
+  // 2 MB per head), at least one head
+#ifndef FA_GROUP_KV_MB
+#define FA_GROUP_KV_MB 64
+#endif
+  const long long kv_head = 2LL * a.Nk * a.D * 2;
+  p.head_group = static_cast<int>(
+      std::max(1LL, std::min<long long>(static_cast<long long>(a.B) * a.H, (static_cast<long long>(FA_GROUP_KV_MB) << 20) / kv_head)));
+#ifdef FA_HEAD_GROUP  // tuning: a fixed head-group size
+  p.head_group = FA_HEAD_GROUP;
+#endif
+  p.tma_out = a.o_fp32 ? 0 : 1;
+#ifdef FA_NO_TMA_OUT  // tuning: per-thread O stores for every tile
+  p.tma_out = 0;
+#endif
   if (a.D == 64) {
-    if (a.fp16) return a.o_fp32 ? launch_t<64, true, true>(a, mq, mk, mv, p, stream) : launch_t<64, true, false>(a, mq, mk, mv, p, stream);
-    return a.o_fp32 ? launch_t<64, false, true>(a, mq, mk, mv, p, stream) : launch_t<64, false, false>(a, mq, mk, mv, p, stream);
+    if (a.fp16) return a.o_fp32 ? launch_t<64, true, true>(a, mq, mk, mv, mo, p, stream) : launch_t<64, true, false>(a, mq, mk, mv, mo, p, stream);
+    return a.o_fp32 ? launch_t<64, false, true>(a, mq, mk, mv, mo, p, stream) : launch_t<64, false, false>(a, mq, mk, mv, mo, p, stream);
   }
-  if (a.fp16) return a.o_fp32 ? launch_t<128, true, true>(a, mq, mk, mv, p, stream) : launch_t<128, true, false>(a, mq, mk, mv, p, stream);
-  return a.o_fp32 ? launch_t<128, false, true>(a, mq, mk, mv, p, stream) : launch_t<128, false, false>(a, mq, mk, mv, p, stream);
+  if (a.fp16) return a.o_fp32 ? launch_t<128, true, true>(a, mq, mk, mv, mo, p, stream) : launch_t<128, true, false>(a, mq, mk, mv, mo, p, stream);
+  return a.o_fp32 ? launch_t<128, false, true>(a, mq, mk, mv, mo, p, stream) : launch_t<128, false, false>(a, mq, mk, mv, mo, p, stream);
 }
 
 }  // namespace fa
