@@ -34,6 +34,8 @@
 // sequences indexed through cu_seqlens (LSE and Drow [H, total]).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "fa_prefill_common.cuh"
 
 namespace fa {
@@ -73,6 +75,7 @@ struct BwdParams {
   float scale, scale_log2;
   int causal;
   int prefix;  // causal only: keys [0, prefix) of a sequence are visible to all of its queries
+  int head_group;  // dense: (b, h) heads whose tiles are ordered together, most work first
 };
 
 // The CTA's (batch item, head, 128-row tile) and its sequence: rows [row0, row0 + L) of the packed
@@ -89,8 +92,14 @@ template <bool kLastFirst>
 __device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, int warp, int lane, int* sh_b, int* sh_t) {
   BwdUnit u;
   if (p.cu == nullptr) {
-    const int bh = static_cast<int>(blockIdx.x / p.num_tiles);
-    const int t = static_cast<int>(blockIdx.x % p.num_tiles);
+    // groups of head_group heads (their streamed tiles fit in L2) one after another; inside a group
+    // the tiles with the most causal work of all its heads first, heads fastest
+    const int bhs = p.B * p.H;
+    const int per_group = p.head_group * p.num_tiles;
+    const int grp = static_cast<int>(blockIdx.x / per_group), w = static_cast<int>(blockIdx.x % per_group);
+    const int gsz = min(p.head_group, bhs - grp * p.head_group);
+    const int bh = grp * p.head_group + w % gsz;
+    const int t = w / gsz;
     u.tile = kLastFirst ? p.num_tiles - 1 - t : t;
     u.b = bh / p.H;
     u.h = bh % p.H;
@@ -756,6 +765,13 @@ int launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   p.causal = a.causal ? 1 : 0;
   p.prefix = a.causal ? a.prefix : 0;
   p.cu = a.cu_seqlens;
+  // about 64 MB of streamed tiles (K and V for dQ, Q and dO for dK/dV) per head group
+  const long long stream_head = 2LL * std::max(a.Nq, a.Nk) * a.D * 2;
+  p.head_group = static_cast<int>(
+      std::max(1LL, std::min<long long>(static_cast<long long>(a.B) * a.H, (64LL << 20) / stream_head)));
+#ifdef FA_BWD_HEAD_GROUP  // tuning: a fixed head-group size
+  p.head_group = FA_BWD_HEAD_GROUP;
+#endif
   if (a.D == 64) {
     if (a.fp16) return a.g_fp32 ? launch_bwd_t<64, true, true>(a, m, p, stream) : launch_bwd_t<64, true, false>(a, m, p, stream);
     return a.g_fp32 ? launch_bwd_t<64, false, true>(a, m, p, stream) : launch_bwd_t<64, false, false>(a, m, p, stream);
