@@ -129,8 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- work unit: (b, h, pair of Q tiles) -----------------------------------------------------
   int b, h, pair;
   if (p.cu == nullptr) {
-    // all pairs of one (b, h) are consecutive, so they run together and share its K/V in L2;
-    // within a head the pair with the most key blocks (causal) goes first
     // Groups of head_group (b, h) heads run one after another, so the K/V of the heads in flight
     // stay in L2; inside a group the pairs with the most key blocks (causal) of all its heads come
     // first, heads fastest, so that the longest units start early and none is left for the end.
