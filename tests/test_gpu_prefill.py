@@ -221,3 +221,37 @@ def test_varlen_full_config():
         h = int(rng.integers(c["H"]))
         ro, rl = oracle.attention_head(qf[s0:s1, h], kf[s0:s1, h], vf[s0:s1, h], c["scale"])
         check(on[s0:s1, h], ln[h, s0:s1], ro, rl, "fp32", f"varlen seq {b} head {h}")
+
+
+def test_partial_last_head_group():
+    """Work units run longest-first inside groups of heads whose K/V take about 64 MB.  With 65536 keys
+    of D = 128 a head's K/V is 32 MB, so two heads form a group and the third head is a group of its
+    own: the last, partial group's units must still all be computed (sampled rows of every head)."""
+    fa = fa_mod()
+    B, N, H, D, dt, scale = 1, 65536, 3, 128, "bf16", 1 / math.sqrt(128)
+    q, k, v = si.dense_qkv(2200, B, N, N, H, D, dt)
+    o, lse = fa.attention(*(to_device(t, dt) for t in (q, k, v)), causal=True, scale=scale, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(clear=True) == 0
+    rows = np.array([0, 1, 255, 256, 30000, N - 257, N - 256, N - 1])
+    for h in range(H):
+        ro, rl = oracle.attention_rows(to_f64(q[0, :, h], dt), to_f64(k[0, :, h], dt), to_f64(v[0, :, h], dt), rows,
+                                       scale, True)
+        check(o[0, :, h].float().cpu().numpy()[rows], lse[0, h].cpu().numpy()[rows], ro, rl, "bf16",
+              f"head {h} of a partial group")
+
+
+@pytest.mark.parametrize("D,dtype", [(64, "bf16"), (128, "fp16")])
+def test_16bit_output_is_fp32_output_rounded(D, dtype):
+    """Full tiles of a 16-bit O are written through shared memory by TMA stores, partial tiles by
+    per-thread stores; both must equal the fp32 output rounded to the 16-bit type, bit for bit."""
+    fa = fa_mod()
+    B, N, H = 2, 700, 3  # tiles 0-4 full, tile 5 partial, per batch item
+    q, k, v = si.dense_qkv(2300 + D, B, N, N, H, D, dtype)
+    args = [to_device(t, dtype) for t in (q, k, v)]
+    for causal in (False, True):
+        o16, l16 = fa.attention(*args, causal=causal, scale=0.1)
+        o32, l32 = fa.attention(*args, causal=causal, scale=0.1, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert torch.equal(o16, o32.to(o16.dtype)), causal
+        assert torch.equal(l16, l32)
