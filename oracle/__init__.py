@@ -8,7 +8,8 @@ library.  The two sides share only the seeded input generator, which holds no at
 Modules:
   attention  -- the materialised definition O = softmax(scale*Q*K^T + mask)*V with LSE, per (b, h);
                 dense, packed-varlen, row-sampled and single-query (decode) forms, the latter also
-                with grouped KV heads, per-sequence cache lengths and over one key shard of a cache.
+                with grouped KV heads, per-sequence cache lengths, over one key shard of a cache and
+                over a paged cache (a page pool addressed through a per-sequence block table).
   online     -- the tiled algorithm in the order the pages give it (Q blocks outside, K/V blocks
                 inside, running max m and running sum l), and the pairwise merge of softmax
                 statistics of key groups, including the split-KV partial/combine form.
@@ -18,7 +19,7 @@ Modules:
 """
 from .attention import (attention_head, attention_dense, attention_varlen, attention_rows,
                         attention_decode, attention_decode_gqa, attention_decode_shard,
-                        padded_key_mask_attention)
+                        attention_decode_paged, padded_key_mask_attention)
 from .online import (tiled_online_attention, group_stats, merge_groups, softmax_by_groups,
                      split_kv_partials, combine_partials)
 from .brute import brute_attention_head
@@ -27,7 +28,7 @@ from .backward import (attention_head_backward, attention_dense_backward, attent
 
 __all__ = [
     "attention_head", "attention_dense", "attention_varlen", "attention_rows", "attention_decode",
-    "attention_decode_gqa", "attention_decode_shard",
+    "attention_decode_gqa", "attention_decode_shard", "attention_decode_paged",
     "padded_key_mask_attention", "tiled_online_attention", "group_stats", "merge_groups",
     "softmax_by_groups", "split_kv_partials", "combine_partials", "brute_attention_head",
     "attention_head_backward", "attention_dense_backward", "attention_varlen_backward",

@@ -215,3 +215,34 @@ def attention_decode_shard(q, k_shard, v_shard, scale: float, key_offset: int, s
     if seqlens_k is not None:
         lens = [min(max(int(L) - key_offset, 0), nk) for L in seqlens_k]
     return attention_decode_gqa(q, k_shard, v_shard, scale, lens)
+
+
+def attention_decode_paged(q, k_pages, v_pages, block_table, scale: float, seqlens_k):
+    """Single-token decode over a paged cache: O [B,1,Hq,Dv] and LSE [B,Hq].
+
+    k_pages/v_pages [P, page_size, Hkv, D] are pools of fixed-size pages of cache rows (row r of page
+    p is one key).  ``block_table`` [B, pages_per_seq] lists, for each batch item, the pool pages that
+    hold its keys in order: entry i holds keys [i * page_size, (i + 1) * page_size).  Batch item b
+    sees its first seqlens_k[b] keys, so only its first ceil(seqlens_k[b] / page_size) entries are
+    read; the rest of the row (and any page no entry names) is never looked at.  The query then
+    attends to the keys gathered in that order exactly as over a contiguous cache with grouped KV
+    heads (query head h reads KV head h // (Hq // Hkv)).
+
+    Reading: "Was FlashAttention bei Transformer-Inference verändert" lists the cache layout among
+    the properties a backend must support without fixing one; a pool of fixed-size pages addressed
+    through a per-sequence table is the plainest layout beside the contiguous one, and it changes
+    only where each key row is read from, not what is computed.
+    """
+    B = q.shape[0]
+    ps = k_pages.shape[1]
+    seqlens_k = [int(L) for L in seqlens_k]
+    lmax = max(seqlens_k + [1])
+    cap = -(-lmax // ps) * ps
+    k_g = np.zeros((B, cap) + k_pages.shape[2:], dtype=np.float64)
+    v_g = np.zeros((B, cap) + v_pages.shape[2:], dtype=np.float64)
+    for b, L in enumerate(seqlens_k):
+        for i in range(-(-L // ps)):
+            page = int(block_table[b][i])
+            k_g[b, i * ps:(i + 1) * ps] = k_pages[page]
+            v_g[b, i * ps:(i + 1) * ps] = v_pages[page]
+    return attention_decode_gqa(q, k_g, v_g, scale, seqlens_k)

@@ -47,6 +47,10 @@ MUTANTS = {
     "bwd_rows_chunk_offset": ("attention.py", "i = np.arange(row_lo, row_hi)[:, None]",
                               "i = np.arange(0, row_hi - row_lo)[:, None]"),
     "bwd_rows_dv_uses_ds": ("backward.py", "dv += pc.T @ do[a:e]", "dv += dsc.T @ do[a:e]"),
+    "paged_table_ignored": ("attention.py", "page = int(block_table[b][i])", "page = i"),
+    "paged_partial_page_dropped": ("attention.py", "for i in range(-(-L // ps)):", "for i in range(L // ps):"),
+    "paged_row_in_page": ("attention.py", "k_g[b, i * ps:(i + 1) * ps] = k_pages[page]",
+                          "k_g[b, i * ps:(i + 1) * ps] = k_pages[page][::-1]"),
 }
 
 

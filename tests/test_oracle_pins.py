@@ -492,6 +492,103 @@ def test_shard_decode_zero_query_closed_form():
 
 
 # ---------------------------------------------------------------------------------------------
+# decode over a paged cache (page pool + per-sequence block table)
+
+
+def _paginate(k, v, ps, rng):
+    """Cut a contiguous cache [B, Nk, Hkv, D] into pages of ps rows, laid into a shuffled pool with a
+    few spare pages; returns the pool, the block table and the spare page indices."""
+    B, Nk = k.shape[:2]
+    npg = -(-Nk // ps)
+    pool_n = B * npg + 3
+    perm = rng.permutation(pool_n)
+    kp = np.full((pool_n, ps) + k.shape[2:], 7.0)
+    vp = np.full((pool_n, ps) + v.shape[2:], 7.0)
+    table = np.zeros((B, npg), dtype=np.int64)
+    for b in range(B):
+        for i in range(npg):
+            page = int(perm[b * npg + i])
+            table[b, i] = page
+            rows = slice(i * ps, min((i + 1) * ps, Nk))
+            kp[page, :rows.stop - rows.start] = k[b, rows]
+            vp[page, :rows.stop - rows.start] = v[b, rows]
+    return kp, vp, table, [int(x) for x in perm[B * npg:]]
+
+
+def test_paged_decode_equals_contiguous_decode():
+    # the same keys in shuffled pages through a table give the contiguous result, bit for bit, for
+    # lengths ending inside a page, at a page edge, at one key, and at zero
+    B, Nk, Hkv, G, D, ps = 5, 37, 2, 3, 8, 8
+    rng = np.random.default_rng(160)
+    q = rnd((B, 1, Hkv * G, D), 161)
+    k, v = rnd((B, Nk, Hkv, D), 162), rnd((B, Nk, Hkv, D), 163)
+    lens = [37, 16, 1, 0, 9]
+    kp, vp, table, _ = _paginate(k, v, ps, rng)
+    o, lse = oracle.attention_decode_paged(q, kp, vp, table, 0.3, lens)
+    o_ref, lse_ref = oracle.attention_decode_gqa(q, k, v, 0.3, lens)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, lse_ref)
+
+
+def test_paged_decode_reads_only_the_named_pages():
+    # table entries past ceil(L / page_size) and pages no entry names may hold anything (here NaN
+    # pages and entry -1): the result is unchanged
+    B, Nk, Hkv, G, D, ps = 3, 24, 1, 2, 8, 4
+    rng = np.random.default_rng(164)
+    q = rnd((B, 1, Hkv * G, D), 165)
+    k, v = rnd((B, Nk, Hkv, D), 166), rnd((B, Nk, Hkv, D), 167)
+    lens = [24, 10, 3]
+    kp, vp, table, spare = _paginate(k, v, ps, rng)
+    o_ref, lse_ref = oracle.attention_decode_paged(q, kp, vp, table, 0.4, lens)
+    kp2, vp2, t2 = kp.copy(), vp.copy(), table.copy()
+    for b, L in enumerate(lens):
+        for i in range(-(-L // ps), t2.shape[1]):
+            kp2[t2[b, i]] = np.nan
+            vp2[t2[b, i]] = np.nan
+            t2[b, i] = -1
+    for page in spare:
+        kp2[page] = np.nan
+        vp2[page] = np.nan
+    o, lse = oracle.attention_decode_paged(q, kp2, vp2, t2, 0.4, lens)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, lse_ref)
+
+
+def test_paged_decode_zero_query_closed_form():
+    # Q = 0: O is the mean of the first L value rows in table order, LSE = ln L
+    B, Hkv, G, D, ps = 3, 2, 2, 8, 4
+    rng = np.random.default_rng(168)
+    pool = 9
+    vp = rnd((pool, ps, Hkv, D), 169)
+    kp = rnd((pool, ps, Hkv, D), 170)
+    table = np.array([rng.permutation(pool)[:3] for _ in range(B)])
+    lens = [12, 5, 1]
+    q = np.zeros((B, 1, Hkv * G, D))
+    o, lse = oracle.attention_decode_paged(q, kp, vp, table, 0.7, lens)
+    for b, L in enumerate(lens):
+        rows = np.concatenate([vp[p] for p in table[b]])[:L]
+        for h in range(Hkv * G):
+            np.testing.assert_allclose(o[b, 0, h], rows[:, h // G].mean(axis=0), rtol=RTOL, atol=1e-14)
+            assert abs(lse[b, h] - math.log(L)) < 1e-13
+
+
+def test_paged_decode_brute_force():
+    # tiny case against scalar evaluation over the keys gathered row by row through the table
+    Hkv, G, D, ps = 1, 2, 3, 2
+    kp, vp = rnd((4, ps, Hkv, D), 171), rnd((4, ps, Hkv, D), 172)
+    table = np.array([[2, 0, 3]])
+    L = 5
+    q = rnd((1, 1, Hkv * G, D), 173)
+    o, lse = oracle.attention_decode_paged(q, kp, vp, table, 0.9, [L])
+    keys = [kp[table[0, j // ps], j % ps, 0] for j in range(L)]
+    vals = [vp[table[0, j // ps], j % ps, 0] for j in range(L)]
+    for h in range(G):
+        ob, lb = oracle.brute_attention_head(q[0, :, h], np.array(keys), np.array(vals), 0.9)
+        np.testing.assert_allclose(o[0, 0, h], ob[0], rtol=1e-12, atol=1e-14)
+        assert abs(lse[0, h] - lb[0]) < 1e-12
+
+
+# ---------------------------------------------------------------------------------------------
 # backward: the derivative of the forward definition
 
 
