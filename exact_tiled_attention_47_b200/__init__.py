@@ -15,11 +15,11 @@ from ._lib import DEBUG_LIB_PATH, LIB_PATH, LibraryMissing, SIGNATURES, load
 
 FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 (FA_OK, FA_ERR_NULL, FA_ERR_DTYPE, FA_ERR_HEADDIM, FA_ERR_SHAPE, FA_ERR_ALIGN, FA_ERR_CU_SEQLENS,
- FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT, FA_ERR_BOUNDS) = range(12)
+ FA_ERR_WORKSPACE, FA_ERR_DEVICE, FA_ERR_LAUNCH, FA_ERR_TIMEOUT, FA_ERR_BOUNDS, FA_ERR_PAGE_TABLE) = range(13)
 FA_BUILD_DEBUG = 1
 
 __all__ = [
-    "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_masked", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_status_string",
+    "fa_fwd", "fa_fwd_prefix", "fa_bwd", "fa_bwd_masked", "fa_bwd_workspace_bytes", "attention_backward", "fa_decode_workspace_bytes", "fa_decode_splitkv", "fa_decode_splitkv_gqa", "fa_decode_splitkv_paged", "decode_paged", "fa_status_string",
     "fa_device_status", "fa_abi_version", "fa_build_flags", "fa_selftest_wait_timeout", "fa_decode_splitkv_noalloc", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_decode_part_bytes", "fa_decode_splitkv_shard", "fa_decode_merge", "decode_sharded", "shard_range", "attention", "decode", "FAError", "LibraryMissing",
     "LIB_PATH", "DEBUG_LIB_PATH", "FA_BF16", "FA_FP16", "FA_FP32", "FA_BUILD_DEBUG",
@@ -133,6 +133,24 @@ def fa_decode_splitkv_gqa(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale,
                                      int(Hkv), int(Nk), int(D), float(scale), int(num_splits), _ptr(seqlens_k),
                                      _ptr(workspace), int(workspace_bytes), _stream(stream), int(in_dtype),
                                      int(o_dtype))
+
+
+def fa_decode_splitkv_paged(q, k_pages, v_pages, block_table, o, lse, B, Hq, Hkv, num_pages, page_size,
+                            pages_per_seq, D, scale, num_splits, seqlens_k, workspace, workspace_bytes=None,
+                            stream=None, in_dtype=None, o_dtype=None) -> int:
+    """Marshal to the C ``fa_decode_splitkv_paged``; returns its status."""
+    lib = load()
+    if in_dtype is None:
+        in_dtype = _dtype_code(q)
+    if o_dtype is None:
+        o_dtype = _dtype_code(o)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.fa_decode_splitkv_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(o),
+                                       _ptr(lse), int(B), int(Hq), int(Hkv), int(num_pages), int(page_size),
+                                       int(pages_per_seq), int(D), float(scale), int(num_splits), _ptr(seqlens_k),
+                                       _ptr(workspace), int(workspace_bytes), _stream(stream), int(in_dtype),
+                                       int(o_dtype))
 
 
 def fa_decode_part_bytes(B, H, D) -> int:
@@ -326,6 +344,32 @@ def decode(q, k_cache, v_cache, scale=None, num_splits=16, out_dtype=None, works
                                    workspace, nb, stream)
     if st != FA_OK:
         raise FAError(st, "fa_decode_splitkv" if Hkv == H and seqlens_k is None else "fa_decode_splitkv_gqa")
+    return o, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens_k=None, scale=None, num_splits=16, out_dtype=None,
+                 workspace=None, stream=None):
+    """O [B,1,Hq,D], LSE [B,Hq] for one query per (batch, head) over a paged cache.
+
+    k_pages/v_pages [num_pages, page_size, Hkv, D]; block_table int32 [B, pages_per_seq] on the device
+    (entry (b, i): the page holding keys [i*page_size, (i+1)*page_size) of batch item b); seqlens_k
+    int32 [B] on the device or None (every table entry in use).
+    """
+    import torch
+    B, _, H, D = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    pages_per_seq = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if workspace is None:
+        workspace = torch.empty(fa_decode_workspace_bytes(B, H, D, num_splits), device=q.device, dtype=torch.uint8)
+    o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
+    lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    st = fa_decode_splitkv_paged(q, k_pages, v_pages, block_table, o, lse, B, H, Hkv, num_pages, page_size,
+                                 pages_per_seq, D, scale, num_splits, seqlens_k, workspace, stream=stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_decode_splitkv_paged")
     return o, lse
 
 

@@ -27,6 +27,8 @@ SIGNATURES = {
                            _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _Z, _P, _I, _I]),
     "fa_decode_splitkv_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _Z, _P, _I, _I]),
+    "fa_decode_splitkv_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _Z, _P,
+                                     _I, _I]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _I, _I]),
     "fa_decode_part_bytes": (_Z, [_I, _I, _I]),
     "fa_decode_splitkv_shard": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _Z, _P, _I]),

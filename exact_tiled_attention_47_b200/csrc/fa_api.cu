@@ -119,6 +119,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_LAUNCH: return "CUDA launch or driver call failed";
     case FA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case FA_ERR_BOUNDS: return "an index check of the debug build caught an access outside its buffer";
+    case FA_ERR_PAGE_TABLE: return "a block-table entry of the paged cache names no page of the pool";
     default: return "unknown status";
   }
 }
@@ -236,7 +237,8 @@ namespace fa {
 
 int decode_checked_launch(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
                           int H, int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k,
-                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream) {
+                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream,
+                          const int* block_table, int pages_per_seq, int page_size, int num_pages) {
   int* status = fa::device_status_ptr();
   if (!status) return FA_ERR_LAUNCH;
   fa::DecodeArgs a;
@@ -261,6 +263,10 @@ int decode_checked_launch(const void* q, const void* k_cache, const void* v_cach
   a.seqlens_k = seqlens_k;
   a.key_offset = key_offset;
   a.Nk_total = Nk_total;
+  a.block_table = block_table;
+  a.pages_per_seq = pages_per_seq;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
   const int e = fa::launch_decode(a, stream);
   if (e != 0) {
     cudaGetLastError();
@@ -311,6 +317,32 @@ int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cach
                           int o_dtype) {
   return decode_impl(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k, workspace,
                      workspace_bytes, stream, in_dtype, o_dtype);
+}
+
+int fa_decode_splitkv_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                            void* o, float* lse, int B, int Hq, int Hkv, int num_pages, int page_size,
+                            int pages_per_seq, int D, float scale, int num_splits, const int* seqlens_k,
+                            void* workspace, size_t workspace_bytes, fa_stream_t stream, int in_dtype,
+                            int o_dtype) {
+  if (!block_table) return FA_ERR_NULL;
+  // page size: a power of two from 16 rows (whole 16-key boxes; 64-key tiles cover whole pages);
+  // pool rows, cache capacity and table size within 32-bit indices
+  if (page_size < 16 || page_size > (1 << 16) || (page_size & (page_size - 1)) != 0) return FA_ERR_SHAPE;
+  if (num_pages < 1 || pages_per_seq < 1 || B < 1) return FA_ERR_SHAPE;
+  if (static_cast<int64_t>(num_pages) * page_size >= (static_cast<int64_t>(1) << 31) ||
+      static_cast<int64_t>(pages_per_seq) * page_size >= (static_cast<int64_t>(1) << 31) ||
+      static_cast<int64_t>(B) * pages_per_seq >= (static_cast<int64_t>(1) << 31))
+    return FA_ERR_SHAPE;
+  const int Nk = pages_per_seq * page_size;
+  if (const int st = decode_check(q, k_pages, v_pages, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                                  workspace, workspace_bytes, false, in_dtype, o_dtype, 0, Nk))
+    return st;
+  if (!fa::aligned(block_table, 4)) return FA_ERR_ALIGN;
+  int dev = -1;
+  if (const int st = fa::check_device(&dev)) return st;
+  return fa::decode_checked_launch(q, k_pages, v_pages, o, lse, B, Hq, Hkv, Nk, D, scale, num_splits, seqlens_k,
+                                   workspace, in_dtype, o_dtype, 0, Nk, reinterpret_cast<cudaStream_t>(stream),
+                                   block_table, pages_per_seq, page_size, num_pages);
 }
 
 size_t fa_decode_part_bytes(int B, int H, int D) {

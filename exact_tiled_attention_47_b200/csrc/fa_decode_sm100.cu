@@ -17,11 +17,18 @@
 //   merge of group statistics of "轻松读懂FlashAttention 上" ("Softmax求解重构") applied to all
 //   splits at once; a query without any key (valid length 0) gets O = 0, LSE = -inf.
 //
+// Paged cache: K and V are pools of pages of 2^page_shift rows and a block table lists each batch
+// item's pages in key order, so key j of batch item b is row table[b][j >> page_shift] *
+// page_size + (j & (page_size - 1)) of the pool.  Both kernels read rows through that mapping;
+// split ranges are then rounded to whole 64-key tiles, so no tile of the tensor-core kernel crosses
+// a page, and each CTA checks the table entries of its range before it reads anything.
+//
 // Key-sharded decode (a cache too long for one GPU cut along the key axis): kernel 1 runs on one
 // shard, seeing the shard's rows as keys [key_offset, key_offset + Nk) of the whole cache, and
 // kernel 2 leaves that shard's fp32 (O, LSE).  The same combine kernel, with other strides, then
 // merges the R shards' results gathered from all ranks (launch_decode_merge): the merge is
 // associative, so combining splits first and shards second gives the softmax over all keys.
+#include <algorithm>
 #include <atomic>
 
 #include "fa_internal.h"
@@ -36,6 +43,7 @@ constexpr int kChunk = 256;
 // A split covers at least this many keys: shorter caches use fewer splits (the rest exit at once),
 // since a CTA's fixed costs (query load, reductions, partial writes) outweigh streaming a few keys.
 constexpr int kMinSplitKeys = 512;
+constexpr int kStatusPageTable = 12;  // FA_ERR_PAGE_TABLE
 
 struct DecParams {
   const void* q;
@@ -52,12 +60,47 @@ struct DecParams {
   int key_offset;   // first key of the whole cache held here
   int Nk_total;     // keys of the whole cache
   float scale_log2;
+  // paged cache (table != nullptr): k and v are pools of num_pages pages of 2^page_shift rows;
+  // table[b * pages_per_seq + i] is the page holding keys [i << page_shift, (i + 1) << page_shift)
+  const int* table;
+  int pages_per_seq, page_shift, num_pages;
 };
+
+// Pool row of key j (counted from the first row held here) of batch item b: the contiguous cache
+// row, or the row the block table maps it to (entries checked beforehand by page_range_ok).
+__device__ __forceinline__ size_t key_row(const DecParams& p, int b, int j) {
+  if (p.table == nullptr) return static_cast<size_t>(b) * p.Nk + j;
+  const int page = __ldg(p.table + static_cast<size_t>(b) * p.pages_per_seq + (j >> p.page_shift));
+  return (static_cast<size_t>(page) << p.page_shift) + (j & ((1 << p.page_shift) - 1));
+}
+
+// Split range [lo, hi) of keys: at least kMinSplitKeys keys per split; on a paged cache rounded up
+// to whole 64-key tiles, so that every tile lies inside one page or covers whole pages.
+__device__ __forceinline__ int split_keys(const DecParams& p, int len) {
+  const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
+  return p.table == nullptr ? per : (per + 63) & ~63;
+}
+
+// True if every block-table entry covering keys [lo, hi) of batch item b names a pool page.
+// Collective over the CTA (every thread must call it); a bad entry is reported as FA_ERR_PAGE_TABLE.
+__device__ __forceinline__ bool page_range_ok(const DecParams& p, int b, int lo, int hi) {
+  if (p.table == nullptr || lo >= hi) return true;
+  bool bad = false;
+  for (int i = (lo >> p.page_shift) + static_cast<int>(threadIdx.x); i <= ((hi - 1) >> p.page_shift);
+       i += blockDim.x) {
+    const int page = __ldg(p.table + static_cast<size_t>(b) * p.pages_per_seq + i);
+    bad |= (page < 0 || page >= p.num_pages);
+  }
+  bad = __syncthreads_or(bad) != 0;
+  if (bad && threadIdx.x == 0) record_status(p.status, kStatusPageTable);
+  return !bad;
+}
 
 // Elements of the buffers a decode kernel touches with plain loads and stores (debug index checks).
 __device__ __forceinline__ long long q_elems(const DecParams& p, int D) { return static_cast<long long>(p.B) * p.H * D; }
 __device__ __forceinline__ long long kv_elems(const DecParams& p, int D) {
-  return static_cast<long long>(p.B) * p.Nk * p.Hkv * D;
+  const long long rows = p.table ? static_cast<long long>(p.num_pages) << p.page_shift : static_cast<long long>(p.B) * p.Nk;
+  return rows * p.Hkv * D;
 }
 __device__ __forceinline__ long long ws_o_elems(const DecParams& p, int D) {
   return static_cast<long long>(p.B) * p.H * p.S * D;
@@ -110,9 +153,10 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
     }
   }
   len = min(max(len - p.key_offset, 0), p.Nk);  // valid keys among the rows held here
-  const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
+  const int per = split_keys(p, len);
   const int lo = min(len, s * per);
-  const int hi = min(len, lo + per);
+  int hi = min(len, lo + per);
+  if (!page_range_ok(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
 
   __shared__ float sc[G][kChunk];
   __shared__ float red_m[4][G];
@@ -146,8 +190,8 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   }
 
   const size_t rs = static_cast<size_t>(p.Hkv) * D;  // elements between consecutive cache rows
-  const T* kb = static_cast<const T*>(p.k) + static_cast<size_t>(b) * p.Nk * rs + hk * D + c * 8;
-  const T* vb = static_cast<const T*>(p.v) + static_cast<size_t>(b) * p.Nk * rs + hk * D + c * 8;
+  const T* kb = static_cast<const T*>(p.k) + hk * D + c * 8;
+  const T* vb = static_cast<const T*>(p.v) + hk * D + c * 8;
 
   float m_run[G], l_part[G], acc[G][8];
 #pragma unroll
@@ -166,9 +210,9 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        if (j < n && idx_ok(p.status, kb + static_cast<size_t>(c0 + j) * rs - static_cast<const T*>(p.k), 8,
-                            kv_elems(p, D))) {
-          load8_stream<kFp16>(kb + static_cast<size_t>(c0 + j) * rs, kf[u]);
+        const size_t row = (j < n) ? key_row(p, b, c0 + j) : 0;
+        if (j < n && idx_ok(p.status, kb + row * rs - static_cast<const T*>(p.k), 8, kv_elems(p, D))) {
+          load8_stream<kFp16>(kb + row * rs, kf[u]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) kf[u][e] = 0.f;
@@ -214,9 +258,9 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        if (j < n && idx_ok(p.status, vb + static_cast<size_t>(c0 + j) * rs - static_cast<const T*>(p.v), 8,
-                            kv_elems(p, D))) {
-          load8_stream<kFp16>(vb + static_cast<size_t>(c0 + j) * rs, vf[u]);
+        const size_t row = (j < n) ? key_row(p, b, c0 + j) : 0;
+        if (j < n && idx_ok(p.status, vb + row * rs - static_cast<const T*>(p.v), 8, kv_elems(p, D))) {
+          load8_stream<kFp16>(vb + row * rs, vf[u]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) vf[u][e] = 0.f;
@@ -377,9 +421,10 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     }
   }
   len = min(max(len - p.key_offset, 0), p.Nk);
-  const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
+  const int per = split_keys(p, len);
   const int lo = min(len, s * per);
-  const int hi = min(len, lo + per);
+  int hi = min(len, lo + per);
+  if (!page_range_ok(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
   auto ws_o = [&](int g) { return p.ws_o + ((static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s) * D; };
   auto ws_l = [&](int g) { return p.ws_lse + (static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s; };
   if (lo >= hi) {  // uniform over the CTA: empty partials
@@ -409,18 +454,25 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
       int issued = 0;
-      const int row0 = b * p.Nk + lo;
+      // a tile is loaded as boxes of `box` rows: one box on a contiguous cache, one box per page on
+      // a paged cache with pages shorter than a tile (boxes past the valid keys are not loaded)
+      const int box = p.table ? min(kMmaTileKeys, 1 << p.page_shift) : kMmaTileKeys;
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % C::kStages;
         if (t >= C::kStages && !mbar_wait(&bars->empty[st], ((t / C::kStages) - 1) & 1, abort_flag, p.status))
           break;
         uint8_t* kdst = smem + st * C::kStageBytes;
-        mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes);
+        const int k0 = lo + t * kMmaTileKeys;
+        const int boxes = min(kMmaTileKeys, hi - k0 + box - 1) / box;
+        mbar_arrive_expect_tx(&bars->full[st], static_cast<uint32_t>(boxes * box * 128 * (D / 64) * 2));
+        for (int i = 0; i < boxes; ++i) {
+          const int row = static_cast<int>(key_row(p, b, k0 + i * box));
 #pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn) {
-          tma_load_3d(&tmap_k, &bars->full[st], kdst + pn * C::kPanelBytes, pn * 64, hk, row0 + t * kMmaTileKeys);
-          tma_load_3d(&tmap_v, &bars->full[st], kdst + C::kTileBytes + pn * C::kPanelBytes, pn * 64, hk,
-                      row0 + t * kMmaTileKeys);
+          for (int pn = 0; pn < D / 64; ++pn) {
+            tma_load_3d(&tmap_k, &bars->full[st], kdst + pn * C::kPanelBytes + i * box * 128, pn * 64, hk, row);
+            tma_load_3d(&tmap_v, &bars->full[st], kdst + C::kTileBytes + pn * C::kPanelBytes + i * box * 128, pn * 64,
+                        hk, row);
+          }
         }
         issued = t + 1;
       }
@@ -475,6 +527,19 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
       // e >= 2 row g + 8
       const int key0 = lo + t * kMmaTileKeys + warp * 16 + 2 * tg;
       const bool tail = (lo + (t + 1) * kMmaTileKeys > hi);
+      if (tail) {
+        // rows of the last tile past the valid keys hold whatever the cache (or a stale stage) holds
+        // there; their P is 0, but 0 * NaN would still reach O, so this warp's V rows there are zeroed
+        const int first_dead = hi - (lo + t * kMmaTileKeys + warp * 16);  // of this warp's 16 rows
+        for (int i = lane; i < 16 * 8 * (D / 64); i += 32) {
+          const int r = i / (8 * (D / 64)), pn = (i / 8) % (D / 64), ch = i % 8;
+          if (r >= first_dead) {
+            const uint32_t a = vb + pn * C::kPanelBytes + (warp * 16 + r) * 128 + ch * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+          }
+        }
+        __syncwarp();
+      }
       uint32_t pa[4];
 #pragma unroll
       for (int r = 0; r < (kHi ? 2 : 1); ++r) {
@@ -528,6 +593,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
           mma16816<kFp16>(o[2 * dt + 1], pa, b2, b3);
         }
       }
+      // the zeroing stores above come before the next asynchronous (TMA) write into the stage
+      if (tail) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->empty[st]);
     }
@@ -665,9 +732,9 @@ void launch_combine(const CombParams& c, bool o_fp32, cudaStream_t stream) {
 template <bool kFp16, int D, int G>
 int launch_mma(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
   CUtensorMap mk, mv;
-  const int rows = a.B * a.Nk;
-  if (!make_tma_map(&mk, a.k, rows, p.Hkv, D, kFp16, kMmaTileKeys) ||
-      !make_tma_map(&mv, a.v, rows, p.Hkv, D, kFp16, kMmaTileKeys))
+  const int rows = p.table ? (p.num_pages << p.page_shift) : a.B * a.Nk;
+  const int box = p.table ? std::min(kMmaTileKeys, 1 << p.page_shift) : kMmaTileKeys;  // as the producer loads
+  if (!make_tma_map(&mk, a.k, rows, p.Hkv, D, kFp16, box) || !make_tma_map(&mv, a.v, rows, p.Hkv, D, kFp16, box))
     return static_cast<int>(cudaErrorInvalidValue);
   auto kern = decode_mma_kernel<kFp16, D, G>;
   // the shared-memory opt-in is a per-device (per-context) attribute of the function: set it once
@@ -685,7 +752,8 @@ template <bool kFp16, int D>
 int launch_decode_t(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
   // Grouped heads: the tensor-core kernel with G = the largest of 16, 8, 4, 2 dividing the group
   // (the TMA maps index rows with 32-bit coordinates); one head per KV head: the CUDA-core kernel.
-  const bool tma_rows_ok = static_cast<long long>(a.B) * a.Nk < (1LL << 31);
+  const long long pool_rows = p.table ? static_cast<long long>(p.num_pages) << p.page_shift : static_cast<long long>(a.B) * a.Nk;
+  const bool tma_rows_ok = pool_rows < (1LL << 31);
   int e = 0;
   if (tma_rows_ok && p.group % 16 == 0) e = launch_mma<kFp16, D, 16>(a, p, stream);
   else if (tma_rows_ok && p.group % 8 == 0) e = launch_mma<kFp16, D, 8>(a, p, stream);
@@ -728,6 +796,11 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.key_offset = a.key_offset;
   p.Nk_total = a.Nk_total > 0 ? a.Nk_total : a.Nk;
   p.scale_log2 = a.scale * kLog2e;
+  p.table = a.block_table;
+  p.pages_per_seq = a.pages_per_seq;
+  p.page_shift = 0;
+  while (a.block_table && (1 << p.page_shift) < a.page_size) ++p.page_shift;
+  p.num_pages = a.num_pages;
   if (a.D == 64) return a.fp16 ? launch_decode_t<true, 64>(a, p, stream) : launch_decode_t<false, 64>(a, p, stream);
   return a.fp16 ? launch_decode_t<true, 128>(a, p, stream) : launch_decode_t<false, 128>(a, p, stream);
 }

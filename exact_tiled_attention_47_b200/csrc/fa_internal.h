@@ -44,6 +44,11 @@ struct DecodeArgs {
   // key_offset + Nk) of a cache of Nk_total keys (0: Nk), and seqlens_k counts keys of the whole cache.
   int key_offset = 0;
   int Nk_total = 0;
+  // Paged cache (block_table != nullptr): k and v are pools of num_pages pages of page_size rows (a
+  // power of two); block_table[b * pages_per_seq + i] is the page holding keys
+  // [i * page_size, (i + 1) * page_size) of batch item b, and Nk = pages_per_seq * page_size.
+  const int* block_table = nullptr;
+  int pages_per_seq = 0, page_size = 0, num_pages = 0;
 };
 
 // Merge of R partial decode results (one per key shard) laid out as R packed blocks of part_floats
@@ -90,7 +95,9 @@ int launch_backward(const BackwardArgs& a, cudaStream_t stream);
 // the split and combine kernels with the per-split partials in ws.  Returns an fa_status.
 int decode_checked_launch(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B,
                           int H, int Hkv, int Nk, int D, float scale, int num_splits, const int* seqlens_k,
-                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream);
+                          void* ws, int in_dtype, int o_dtype, int key_offset, int Nk_total, cudaStream_t stream,
+                          const int* block_table = nullptr, int pages_per_seq = 0, int page_size = 0,
+                          int num_pages = 0);
 // The boundary's decode argument checks for a workspace of fixed capacity (no caller pointer).
 int decode_check_fixed(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse, int B, int H,
                        int Nk, int D, float scale, int num_splits, size_t capacity, int in_dtype, int o_dtype);

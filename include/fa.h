@@ -57,8 +57,10 @@ typedef enum {
   FA_ERR_DEVICE = 8,      /* no CUDA device, or the current device is not sm_100             */
   FA_ERR_LAUNCH = 9,      /* a CUDA launch or driver call failed                              */
   FA_ERR_TIMEOUT = 10,    /* a bounded wait inside a kernel ran out (device-detected)         */
-  FA_ERR_BOUNDS = 11      /* debug builds only: an index check caught an access outside its
+  FA_ERR_BOUNDS = 11,     /* debug builds only: an index check caught an access outside its
                              buffer (device-detected; the access was skipped)                  */
+  FA_ERR_PAGE_TABLE = 12  /* a paged-cache block-table entry names no pool page
+                             (device-detected; see fa_decode_splitkv_paged)                     */
 } fa_status;
 
 /*
@@ -210,6 +212,37 @@ int fa_decode_splitkv_gqa(const void* q, const void* k_cache, const void* v_cach
                           int B, int Hq, int Hkv, int Nk, int D, float scale, int num_splits,
                           const int* seqlens_k, void* workspace, size_t workspace_bytes,
                           fa_stream_t stream, int in_dtype, int o_dtype);
+
+/*
+ * fa_decode_splitkv_paged -- fa_decode_splitkv_gqa over a paged cache: a pool of fixed-size pages
+ * of cache rows and a per-sequence table of page indices.
+ *
+ * Passage: as fa_decode_splitkv_gqa ("Was FlashAttention bei Transformer-Inference verändert":
+ * whether a backend supports the cache layout).  A page pool read through a block table is the
+ * layout a serving runtime gets when it grows each sequence's cache by whole pages; it changes
+ * where each key row is read from, not what is computed.
+ *
+ * k_pages, v_pages [num_pages, page_size, Hkv, D] (16-byte aligned); row r of page p is one key.
+ * block_table: device int32 [B, pages_per_seq] (4-byte aligned), row-major; entry (b, i) is the page
+ * holding keys [i * page_size, (i + 1) * page_size) of batch item b.  seqlens_k: device int32[B] or
+ * NULL: batch item b sees its first seqlens_k[b] keys (all pages_per_seq * page_size when NULL);
+ * only the first ceil(seqlens_k[b] / page_size) entries of its table row are read, and nothing of a
+ * page beyond the valid keys reaches the result (it may hold anything, NaN included).
+ * page_size: a power of two, 16 <= page_size <= 65536; num_pages * page_size, pages_per_seq *
+ * page_size and B * pages_per_seq below 2^31 (else FA_ERR_SHAPE).  q, o, lse, workspace, num_splits,
+ * dtypes: as fa_decode_splitkv_gqa, with Nk = pages_per_seq * page_size (split ranges are rounded to
+ * whole 64-key tiles).  Errors as fa_decode_splitkv_gqa, plus FA_ERR_NULL for a NULL block_table and
+ * FA_ERR_ALIGN for a misaligned one.  A table entry outside [0, num_pages) that a batch item needs is
+ * detected on the device: nothing outside the pool is read, the split-KV range holding it
+ * contributes nothing (so that item's O and LSE are not meaningful) and the device status becomes
+ * FA_ERR_PAGE_TABLE.  The function computed is fa_decode_splitkv_gqa's over the rows gathered in
+ * table order.
+ */
+int fa_decode_splitkv_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                            void* o, float* lse, int B, int Hq, int Hkv, int num_pages, int page_size,
+                            int pages_per_seq, int D, float scale, int num_splits, const int* seqlens_k,
+                            void* workspace, size_t workspace_bytes, fa_stream_t stream, int in_dtype,
+                            int o_dtype);
 
 /*
  * fa_decode_part_bytes -- size of one key shard's partial decode result (see

@@ -25,7 +25,7 @@ int main(int argc, char** argv) {
 
   CHECK(fa_abi_version() == 1);
   CHECK(fa_build_flags() == 0 || fa_build_flags() == FA_BUILD_DEBUG);
-  for (code = FA_OK; code <= FA_ERR_BOUNDS; ++code) CHECK(strcmp(fa_status_string(code), "unknown status") != 0);
+  for (code = FA_OK; code <= FA_ERR_PAGE_TABLE; ++code) CHECK(strcmp(fa_status_string(code), "unknown status") != 0);
   CHECK(strcmp(fa_status_string(FA_OK), fa_status_string(FA_ERR_NULL)) != 0);
   CHECK(strcmp(fa_status_string(-1), "unknown status") == 0);
 
@@ -42,11 +42,17 @@ int main(int argc, char** argv) {
   CHECK(fa_decode_merge(AF, 0, 2, 8, 128, A, AF, NULL, FA_BF16) == FA_ERR_SHAPE);
   CHECK(fa_decode_splitkv_shard(A, A, A, AF, 2, 8, 2, 64, 65, 128, 128, 0.1f, 4, NULL, A, 1 << 20, NULL, FA_BF16) ==
         FA_ERR_SHAPE);
+  CHECK(fa_decode_splitkv_paged(A, A, A, NULL, A, AF, 2, 8, 2, 32, 64, 4, 128, 0.1f, 4, NULL, A, 1 << 20, NULL,
+                                FA_BF16, FA_BF16) == FA_ERR_NULL);
+  CHECK(fa_decode_splitkv_paged(A, A, A, (const int*)A, A, AF, 2, 8, 2, 32, 48, 4, 128, 0.1f, 4, NULL, A, 1 << 20,
+                                NULL, FA_BF16, FA_BF16) == FA_ERR_SHAPE);
   CHECK(fa_device_status(NULL, 0) == FA_ERR_NULL);
 
   if (no_device) { /* every argument valid: only the device check fails, nothing is launched */
     CHECK(fa_fwd(A, A, A, A, AF, 1, 1, 128, 128, 64, 0.125f, 1, NULL, NULL, FA_BF16, FA_FP32) == FA_ERR_DEVICE);
     CHECK(fa_decode_merge(AF, 2, 2, 8, 128, A, AF, NULL, FA_FP32) == FA_ERR_DEVICE);
+    CHECK(fa_decode_splitkv_paged(A, A, A, (const int*)A, A, AF, 2, 8, 2, 32, 16, 4, 128, 0.1f, 4, NULL, A, 1 << 20,
+                                  NULL, FA_BF16, FA_FP32) == FA_ERR_DEVICE);
     CHECK(fa_device_status(&st, 0) == FA_ERR_DEVICE);
   }
   printf(fails ? "c_abi_check: %d failure(s)\n" : "c_abi_check: ok\n", fails);

@@ -85,3 +85,29 @@ class Guarded:
         lo = self.raw[:GUARD_BYTES]
         hi = self.raw[GUARD_BYTES + self.nbytes:]
         return bool(torch.all(lo == GUARD_FILL).item() and torch.all(hi == GUARD_FILL).item())
+
+
+NAN_BITS = {"bf16": 0x7FC0, "fp16": 0x7E00}  # a quiet NaN of each 16-bit type
+
+
+def paginate(k_bits, v_bits, lens, ps, dtype, seed, spare=3, shuffle=True):
+    """Pool [P, ps, Hkv, D] (16-bit patterns) and block table [B, pages_per_seq] (int32) holding the
+    contiguous cache's valid rows; NaN everywhere else, -1 in the table entries no item needs."""
+    B, Nk, Hkv, D = k_bits.shape
+    pps = -(-Nk // ps)
+    need = [-(-int(L) // ps) for L in lens]
+    P = sum(need) + spare
+    perm = np.random.default_rng(seed).permutation(P) if shuffle else np.arange(P)
+    kp = np.full((P, ps, Hkv, D), NAN_BITS[dtype], dtype=np.uint16)
+    vp = np.full((P, ps, Hkv, D), NAN_BITS[dtype], dtype=np.uint16)
+    table = np.full((B, pps), -1, dtype=np.int32)
+    t = 0
+    for b, L in enumerate(lens):
+        for i in range(need[b]):
+            page = int(perm[t])
+            t += 1
+            table[b, i] = page
+            n = min(ps, int(L) - i * ps)
+            kp[page, :n] = k_bits[b, i * ps:i * ps + n]
+            vp[page, :n] = v_bits[b, i * ps:i * ps + n]
+    return kp, vp, table

@@ -53,11 +53,11 @@ def test_binding_names_match_c_names():
 def test_abi_version_and_status_strings(lib):
     assert fa.fa_abi_version() == 1
     seen = set()
-    for code in range(12):
+    for code in range(13):
         s = fa.fa_status_string(code)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 12
+    assert len(seen) == 13
     assert fa.fa_status_string(999) == "unknown status"
     assert fa.fa_build_flags() == 0  # the release library
 
@@ -163,6 +163,29 @@ def test_decode_gqa_validation_codes(lib):
     assert gqa(wsb=need - 1) == fa.FA_ERR_WORKSPACE
 
 
+def _paged(lib, table=A, npg=32, ps=64, pps=4, B=2, Hq=8, Hkv=2, sl=None, ws=A, wsb=1 << 20, q=A, kp=A, D=128):
+    return lib.fa_decode_splitkv_paged(q, kp, A, table, A, A, B, Hq, Hkv, npg, ps, pps, D, 0.1, 4, sl, ws, wsb,
+                                       None, 0, 0)
+
+
+def test_decode_paged_validation_codes(lib):
+    assert _paged(lib, table=None) == fa.FA_ERR_NULL
+    assert _paged(lib, q=None) == fa.FA_ERR_NULL
+    for ps in (8, 48, 96, 1 << 17):        # page size: a power of two from 16 to 65536
+        assert _paged(lib, ps=ps) == fa.FA_ERR_SHAPE, ps
+    assert _paged(lib, npg=0) == fa.FA_ERR_SHAPE
+    assert _paged(lib, pps=0) == fa.FA_ERR_SHAPE
+    assert _paged(lib, npg=1 << 25, ps=64) == fa.FA_ERR_SHAPE    # pool rows reach 2^31
+    assert _paged(lib, pps=1 << 25, ps=64) == fa.FA_ERR_SHAPE    # capacity reaches 2^31
+    assert _paged(lib, Hkv=3) == fa.FA_ERR_SHAPE
+    assert _paged(lib, D=96) == fa.FA_ERR_HEADDIM
+    assert _paged(lib, kp=A + 8) == fa.FA_ERR_ALIGN
+    assert _paged(lib, table=A + 2) == fa.FA_ERR_ALIGN
+    assert _paged(lib, sl=A + 2) == fa.FA_ERR_ALIGN
+    need = fa.fa_decode_workspace_bytes(2, 8, 128, 4)
+    assert _paged(lib, wsb=need - 1) == fa.FA_ERR_WORKSPACE
+
+
 def _shard(lib, part=A, q=A, Nk=64, off=0, tot=128, sl=None, ws=A, wsb=1 << 20, in_dtype=0):
     return lib.fa_decode_splitkv_shard(q, A, A, part, 2, 8, 2, Nk, off, tot, 128, 0.1, 4, sl, ws, wsb, None, in_dtype)
 
@@ -261,6 +284,8 @@ def test_no_device_is_reported(lib):
     assert lib.fa_bwd_masked(A, A, A, A, A, A, A, A, A, 2, 1, 300, 300, 64, 0.125, 1, 7, A, A, 1 << 20, None, 0,
                              0) == fa.FA_ERR_DEVICE
     assert lib.fa_decode_splitkv_gqa(A, A, A, A, A, 2, 8, 2, 64, 128, 0.1, 4, A, A, 1 << 20, None, 0, 0) == fa.FA_ERR_DEVICE
+    assert _paged(lib) == fa.FA_ERR_DEVICE
+    assert _paged(lib, ps=16, sl=A) == fa.FA_ERR_DEVICE
     assert _shard(lib) == fa.FA_ERR_DEVICE
     assert _shard(lib, off=64, sl=A) == fa.FA_ERR_DEVICE
     assert _merge(lib) == fa.FA_ERR_DEVICE

@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 import seeded_inputs as si
-from parity import check, to_device, to_f64
+from parity import check, paginate, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -129,6 +129,23 @@ def test_debug_decode(use_debug, Hq, Hkv, D, S, lens):
     o_ref, lse_ref = oracle.attention_decode_gqa(to_f64(q, "bf16"), to_f64(k, "bf16"), to_f64(v, "bf16"),
                                                  1 / math.sqrt(D), lens)
     check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "fp32", "debug decode")
+
+
+@pytest.mark.parametrize("Hq,Hkv,ps", [(16, 4, 16), (4, 4, 128)])
+def test_debug_paged_decode(use_debug, Hq, Hkv, ps):
+    fa = use_debug
+    B, D, S = 3, 64, 4
+    lens = [1000, 0, 65]
+    Nk = -(-max(lens) // ps) * ps
+    q, k, v = si.decode_gqa_inputs(8700 + ps, B, Nk, Hq, Hkv, D, "bf16")
+    kp, vp, table = paginate(k, v, lens, ps, "bf16", 8701)
+    o, lse = fa.decode_paged(*(to_device(t, "bf16") for t in (q, kp, vp)), torch.from_numpy(table).cuda(),
+                             torch.tensor(lens, dtype=torch.int32, device="cuda"), num_splits=S,
+                             out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_decode_paged(to_f64(q, "bf16"), to_f64(kp, "bf16"), to_f64(vp, "bf16"), table,
+                                                   1 / math.sqrt(D), lens)
+    check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "fp32", "debug paged decode")
 
 
 def test_debug_shard_and_merge(use_debug):

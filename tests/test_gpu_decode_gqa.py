@@ -110,3 +110,27 @@ def test_gqa_full_config_sampled():
         o_ref, lse_ref = oracle.attention_decode_gqa(to_f64(q[b:b + 1], "bf16"), to_f64(k[b:b + 1], "bf16"),
                                                      to_f64(v[b:b + 1], "bf16"), c["scale"], [int(lens[b])])
         check(on[b:b + 1], ln[b:b + 1], o_ref, lse_ref, "fp32", f"decode_gqa item {b} len {lens[b]}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,dtype", [(16, 4, 64, "bf16"), (8, 1, 128, "fp16"), (6, 6, 64, "bf16")])
+def test_nan_past_the_valid_length_does_not_reach_o(Hq, Hkv, D, dtype):
+    # cache rows past an item's valid length may hold anything, NaN included (capacity never
+    # written); the last 64-key tile of the tensor-core kernel loads some of them, so their value
+    # rows must not enter P V even with P = 0
+    import exact_tiled_attention_47_b200 as fa
+    B, Nk, S = 3, 1000, 4
+    lens = [999, 500, 77]
+    q, k, v = si.decode_gqa_inputs(990 + Hq, B, Nk, Hq, Hkv, D, dtype)
+    nan = {"bf16": 0x7FC0, "fp16": 0x7E00}[dtype]
+    k2, v2 = k.copy(), v.copy()
+    for b, L in enumerate(lens):
+        k2[b, L:] = nan
+        v2[b, L:] = nan
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    o, lse = fa.decode(to_device(q, dtype), to_device(k2, dtype), to_device(v2, dtype), num_splits=S,
+                       out_dtype=torch.float32, seqlens_k=sl)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(clear=True) == 0
+    o_ref, lse_ref = oracle.attention_decode_gqa(to_f64(q, dtype), to_f64(k, dtype), to_f64(v, dtype),
+                                                 1 / math.sqrt(D), lens)
+    check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "fp32", f"NaN past the lengths, Hq{Hq} Hkv{Hkv}")

@@ -15,7 +15,7 @@ import pytest
 
 import oracle
 import seeded_inputs as si
-from parity import Guarded, check, to_device, to_f64, torch_dtype
+from parity import Guarded, check, paginate, to_device, to_f64, torch_dtype
 
 pytestmark = pytest.mark.gpu
 
@@ -124,6 +124,30 @@ def test_decode_writes_stay_inside(case):
     finish(fa, og, lg, wg)
     o_ref, lse_ref = oracle.attention_decode_gqa(to_f64(q, dtype), to_f64(k, dtype), to_f64(v, dtype), scale, lens)
     check(og.t.float().cpu().numpy(), lg.t.cpu().numpy(), o_ref, lse_ref, out, f"guarded decode {case}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,ps", [(16, 4, 16), (6, 6, 64)])
+def test_paged_decode_writes_stay_inside(Hq, Hkv, ps):
+    fa = fa_mod()
+    B, D, S, dtype = 3, 128, 8, "bf16"
+    lens = [700, 1, 129]
+    Nk = -(-max(lens) // ps) * ps
+    scale = 1 / math.sqrt(D)
+    q, k, v = si.decode_gqa_inputs(7700 + ps, B, Nk, Hq, Hkv, D, dtype)
+    kp, vp, table = paginate(k, v, lens, ps, dtype, 7701)
+    og = Guarded((B, 1, Hq, D), torch.float32)
+    lg = Guarded((B, Hq), torch.float32)
+    nb = fa.fa_decode_workspace_bytes(B, Hq, D, S)
+    wg = Guarded((nb,), torch.uint8)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    st = fa.fa_decode_splitkv_paged(to_device(q, dtype), to_device(kp, dtype), to_device(vp, dtype),
+                                    torch.from_numpy(table).cuda(), og.t, lg.t, B, Hq, Hkv, kp.shape[0], ps,
+                                    table.shape[1], D, scale, S, sl, wg.t, nb)
+    assert st == fa.FA_OK, fa.fa_status_string(st)
+    finish(fa, og, lg, wg)
+    o_ref, lse_ref = oracle.attention_decode_paged(to_f64(q, dtype), to_f64(kp, dtype), to_f64(vp, dtype), table,
+                                                   scale, lens)
+    check(og.t.cpu().numpy(), lg.t.cpu().numpy(), o_ref, lse_ref, "fp32", f"guarded paged decode page {ps}")
 
 
 def test_shard_blocks_and_merge_stay_inside():
