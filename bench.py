@@ -278,11 +278,11 @@ def add_token_rates(line, world):
         dec = line.get("decode") or {}
         if dec.get("ms_per_step"):
             dec["tokens_per_s"] = rate(dec["config"]["B"] * world, dec["ms_per_step"])
-        for key in ("gqa", "sharded"):
+        for key in ("gqa", "paged", "sharded"):
             sub = dec.get(key) or {}
             if sub.get("ms_per_step"):
                 # the sharded cache is one problem split over the ranks: its B sequences per step
-                n = sub["config"]["B"] * (world if key == "gqa" else 1)
+                n = sub["config"]["B"] * (world if key != "sharded" else 1)
                 sub["tokens_per_s"] = rate(n, sub["ms_per_step"])
     except (KeyError, TypeError, ZeroDivisionError):
         pass
@@ -781,7 +781,55 @@ def main():
                                    "traffic": measured_traffic("decode_gqa", kv_g),
                                    "algorithmic_bytes_per_step": alg_g},
                       "gpu_launches": 2 * dsteps}
-        del qg, kg, vg, og, lg_, wsg, sl
+
+        # the same workload over a paged cache: the valid rows of each sequence in pages of 16 rows
+        # at seeded pool positions (the pool is built on the device from the contiguous cache)
+        pc = si.CONFIGS["decode_paged"]
+        ps = pc["page_size"]
+        need = [(int(L) + ps - 1) // ps for L in lens]
+        n_pages = sum(need)
+        pps = (Nkg + ps - 1) // ps
+        perm = np.random.default_rng(rank_seed(pc["seed"], rank)).permutation(n_pages)
+        table = np.full((Bg, pps), -1, dtype=np.int32)
+        kp = torch.empty((n_pages, ps, Hkv, Dg), dtype=torch.bfloat16, device=dev)
+        vp = torch.empty_like(kp)
+        t0 = 0
+        for b, n in enumerate(need):
+            pages = perm[t0:t0 + n]
+            t0 += n
+            table[b, :n] = pages
+            idx = torch.from_numpy(pages).to(dev)
+            kp[idx] = kg[b, :n * ps].view(n, ps, Hkv, Dg)
+            vp[idx] = vg[b, :n * ps].view(n, ps, Hkv, Dg)
+        del kg, vg
+        torch.cuda.empty_cache()
+        tbl = torch.from_numpy(table).to(dev)
+
+        def pstep():
+            st = fa.fa_decode_splitkv_paged(qg, kp, vp, tbl, og, lg_, Bg, Hq, Hkv, n_pages, ps, pps, Dg, g["scale"],
+                                            Sg, sl, wsg, wsbg, stream)
+            if st:
+                raise fa.FAError(st, "fa_decode_splitkv_paged")
+
+        for _ in range(args.warmup):
+            pstep()
+        ms_p = timed(pstep, dsteps, stream, dist)
+        if fa.fa_device_status(clear=True) != 0:
+            raise RuntimeError("device status set during the timed paged decode run")
+        alg_p = alg_g + 4 * n_pages  # plus the table entries read
+        gbs_p = alg_p / (ms_p / dsteps * 1e-3) / 1e9
+        dec["paged"] = {"metric": "paged decode HBM GB/s", "value": gbs_p * world, "unit": "GB/s",
+                        "ms_per_step": ms_p / dsteps, "steps": dsteps,
+                        "config": {"workload": "decode_paged", "B": Bg, "Hq": Hq, "Hkv": Hkv, "D": Dg,
+                                   "num_splits": Sg, "lengths": f"U{{{g['len_lo']}..{g['len_hi']}}}",
+                                   "page_size": ps, "pages": n_pages, "pages_per_seq": pps,
+                                   "page_order": "seeded permutation of the pool", "valid_kv_bytes": kv_g},
+                        "roofline": {"bound": "hbm", "achieved": gbs_p, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs_p / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy",
+                                     "traffic": measured_traffic("decode_paged", kv_g),
+                                     "algorithmic_bytes_per_step": alg_p},
+                        "gpu_launches": 2 * dsteps}
+        del qg, kp, vp, tbl, og, lg_, wsg, sl
         torch.cuda.empty_cache()
 
     # ---------------- CPU baseline (oracle) ----------------

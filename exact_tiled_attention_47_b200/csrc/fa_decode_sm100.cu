@@ -67,24 +67,31 @@ struct DecParams {
 };
 
 // Pool row of key j (counted from the first row held here) of batch item b: the contiguous cache
-// row, or the row the block table maps it to (entries checked beforehand by page_range_ok).
+// row, or the row the block table maps it to (entries checked beforehand by page_range_ok).  The
+// layout is a template parameter of the kernels, so the contiguous ones carry no table code.
+template <bool kPaged>
 __device__ __forceinline__ size_t key_row(const DecParams& p, int b, int j) {
-  if (p.table == nullptr) return static_cast<size_t>(b) * p.Nk + j;
-  const int page = __ldg(p.table + static_cast<size_t>(b) * p.pages_per_seq + (j >> p.page_shift));
-  return (static_cast<size_t>(page) << p.page_shift) + (j & ((1 << p.page_shift) - 1));
+  if constexpr (!kPaged) {
+    return static_cast<size_t>(b) * p.Nk + j;
+  } else {
+    const int page = __ldg(p.table + static_cast<size_t>(b) * p.pages_per_seq + (j >> p.page_shift));
+    return (static_cast<size_t>(page) << p.page_shift) + (j & ((1 << p.page_shift) - 1));
+  }
 }
 
 // Split range [lo, hi) of keys: at least kMinSplitKeys keys per split; on a paged cache rounded up
 // to whole 64-key tiles, so that every tile lies inside one page or covers whole pages.
+template <bool kPaged>
 __device__ __forceinline__ int split_keys(const DecParams& p, int len) {
   const int per = max((len + p.S - 1) / p.S, kMinSplitKeys);
-  return p.table == nullptr ? per : (per + 63) & ~63;
+  return kPaged ? (per + 63) & ~63 : per;
 }
 
 // True if every block-table entry covering keys [lo, hi) of batch item b names a pool page.
 // Collective over the CTA (every thread must call it); a bad entry is reported as FA_ERR_PAGE_TABLE.
+template <bool kPaged>
 __device__ __forceinline__ bool page_range_ok(const DecParams& p, int b, int lo, int hi) {
-  if (p.table == nullptr || lo >= hi) return true;
+  if (!kPaged || lo >= hi) return true;
   bool bad = false;
   for (int i = (lo >> p.page_shift) + static_cast<int>(threadIdx.x); i <= ((hi - 1) >> p.page_shift);
        i += blockDim.x) {
@@ -129,7 +136,7 @@ __device__ __forceinline__ void load8_stream(const void* ptr, float (&f)[8]) {
   f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
 
-template <bool kFp16, int D, int G>
+template <bool kFp16, int D, int G, bool kPaged>
 __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_kernel(const DecParams p) {
   using T = uint16_t;
   constexpr int LPK = D / 8;       // lanes sharing one key row (16-byte slice each)
@@ -153,10 +160,10 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
     }
   }
   len = min(max(len - p.key_offset, 0), p.Nk);  // valid keys among the rows held here
-  const int per = split_keys(p, len);
+  const int per = split_keys<kPaged>(p, len);
   const int lo = min(len, s * per);
   int hi = min(len, lo + per);
-  if (!page_range_ok(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
+  if (!page_range_ok<kPaged>(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
 
   __shared__ float sc[G][kChunk];
   __shared__ float red_m[4][G];
@@ -190,8 +197,19 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
   }
 
   const size_t rs = static_cast<size_t>(p.Hkv) * D;  // elements between consecutive cache rows
-  const T* kb = static_cast<const T*>(p.k) + hk * D + c * 8;
-  const T* vb = static_cast<const T*>(p.v) + hk * D + c * 8;
+  // contiguous: the batch item's rows from here; paged: rows of the pool (through the table)
+  const size_t b_off = kPaged ? 0 : static_cast<size_t>(b) * p.Nk * rs;
+  const T* kb = static_cast<const T*>(p.k) + b_off + hk * D + c * 8;
+  const T* vb = static_cast<const T*>(p.v) + b_off + hk * D + c * 8;
+  // Element offset of key c0 + j of the current chunk: an affine function on a contiguous cache (the
+  // compiler then keeps all UNR loads in flight); on a paged cache the pool row of every key of the
+  // chunk is staged in shared memory once per chunk, so the key loop reads it with one shared load
+  // (a table lookup in front of every key load cost two thirds of the bandwidth).
+  __shared__ int s_row[kPaged ? kChunk : 1];
+  auto row_off = [&](int c0, int j) -> size_t {
+    if constexpr (kPaged) return static_cast<size_t>(s_row[j]) * rs;
+    else return static_cast<size_t>(c0 + j) * rs;
+  };
 
   float m_run[G], l_part[G], acc[G][8];
 #pragma unroll
@@ -204,15 +222,19 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 
   for (int c0 = lo; c0 < hi; c0 += kChunk) {
     const int n = min(kChunk, hi - c0);
+    if constexpr (kPaged) {  // pool rows of the chunk's keys (their table entries were checked)
+      for (int j = tid; j < n; j += kDecThreads) s_row[j] = static_cast<int>(key_row<true>(p, b, c0 + j));
+      __syncthreads();
+    }
     // scores of this chunk: each K row slice is loaded once for the G queries
     for (int j0 = warp * KPW; j0 < n; j0 += UNR * KPB) {
       float kf[UNR][8];
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        const size_t row = (j < n) ? key_row(p, b, c0 + j) : 0;
-        if (j < n && idx_ok(p.status, kb + row * rs - static_cast<const T*>(p.k), 8, kv_elems(p, D))) {
-          load8_stream<kFp16>(kb + row * rs, kf[u]);
+        const size_t off = (kPaged && j >= n) ? 0 : row_off(c0, j);
+        if (j < n && idx_ok(p.status, kb + off - static_cast<const T*>(p.k), 8, kv_elems(p, D))) {
+          load8_stream<kFp16>(kb + off, kf[u]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) kf[u][e] = 0.f;
@@ -258,9 +280,9 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 4 ? 1 : 4)) decode_split_ke
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int j = j0 + u * KPB + kk;
-        const size_t row = (j < n) ? key_row(p, b, c0 + j) : 0;
-        if (j < n && idx_ok(p.status, vb + row * rs - static_cast<const T*>(p.v), 8, kv_elems(p, D))) {
-          load8_stream<kFp16>(vb + row * rs, vf[u]);
+        const size_t off = (kPaged && j >= n) ? 0 : row_off(c0, j);
+        if (j < n && idx_ok(p.status, vb + off - static_cast<const T*>(p.v), 8, kv_elems(p, D))) {
+          load8_stream<kFp16>(vb + off, vf[u]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) vf[u][e] = 0.f;
@@ -391,7 +413,7 @@ __device__ __forceinline__ uint32_t swz_off(int row, int col) {
                                ((((col & 63) >> 3) ^ (row & 7)) << 4));
 }
 
-template <bool kFp16, int D, int G>
+template <bool kFp16, int D, int G, bool kPaged>
 __global__ void __launch_bounds__(kMmaThreads, 2)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                       const DecParams p) {
@@ -421,10 +443,10 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     }
   }
   len = min(max(len - p.key_offset, 0), p.Nk);
-  const int per = split_keys(p, len);
+  const int per = split_keys<kPaged>(p, len);
   const int lo = min(len, s * per);
   int hi = min(len, lo + per);
-  if (!page_range_ok(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
+  if (!page_range_ok<kPaged>(p, b, lo, hi)) hi = lo;  // a bad table entry: the range contributes nothing
   auto ws_o = [&](int g) { return p.ws_o + ((static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s) * D; };
   auto ws_l = [&](int g) { return p.ws_lse + (static_cast<size_t>(b) * p.H + hq0 + g) * p.S + s; };
   if (lo >= hi) {  // uniform over the CTA: empty partials
@@ -456,7 +478,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
       int issued = 0;
       // a tile is loaded as boxes of `box` rows: one box on a contiguous cache, one box per page on
       // a paged cache with pages shorter than a tile (boxes past the valid keys are not loaded)
-      const int box = p.table ? min(kMmaTileKeys, 1 << p.page_shift) : kMmaTileKeys;
+      const int box = kPaged ? min(kMmaTileKeys, 1 << p.page_shift) : kMmaTileKeys;
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % C::kStages;
         if (t >= C::kStages && !mbar_wait(&bars->empty[st], ((t / C::kStages) - 1) & 1, abort_flag, p.status))
@@ -466,7 +488,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
         const int boxes = min(kMmaTileKeys, hi - k0 + box - 1) / box;
         mbar_arrive_expect_tx(&bars->full[st], static_cast<uint32_t>(boxes * box * 128 * (D / 64) * 2));
         for (int i = 0; i < boxes; ++i) {
-          const int row = static_cast<int>(key_row(p, b, k0 + i * box));
+          const int row = static_cast<int>(key_row<kPaged>(p, b, k0 + i * box));
 #pragma unroll
           for (int pn = 0; pn < D / 64; ++pn) {
             tma_load_3d(&tmap_k, &bars->full[st], kdst + pn * C::kPanelBytes + i * box * 128, pn * 64, hk, row);
@@ -717,7 +739,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const CombParams p)
 
 template <bool kFp16, int D, int G>
 void launch_split(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
-  decode_split_kernel<kFp16, D, G><<<dim3(p.Hkv * (p.group / G), a.S, a.B), kDecThreads, 0, stream>>>(p);
+  const dim3 grid(p.Hkv * (p.group / G), a.S, a.B);
+  if (p.table)
+    decode_split_kernel<kFp16, D, G, true><<<grid, kDecThreads, 0, stream>>>(p);
+  else
+    decode_split_kernel<kFp16, D, G, false><<<grid, kDecThreads, 0, stream>>>(p);
 }
 
 template <bool kFp16, int D>
@@ -736,12 +762,17 @@ int launch_mma(const DecodeArgs& a, const DecParams& p, cudaStream_t stream) {
   const int box = p.table ? std::min(kMmaTileKeys, 1 << p.page_shift) : kMmaTileKeys;  // as the producer loads
   if (!make_tma_map(&mk, a.k, rows, p.Hkv, D, kFp16, box) || !make_tma_map(&mv, a.v, rows, p.Hkv, D, kFp16, box))
     return static_cast<int>(cudaErrorInvalidValue);
-  auto kern = decode_mma_kernel<kFp16, D, G>;
+  auto kern = p.table ? decode_mma_kernel<kFp16, D, G, true> : decode_mma_kernel<kFp16, D, G, false>;
   // the shared-memory opt-in is a per-device (per-context) attribute of the function: set it once
+  // (for both layouts' instantiations)
   static PerContext<int> configured;
   int unused = 0;
   const int ce = configured.get(&unused, [&](int*) {
-    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MmaCfg<D>::kSmemBytes));
+    for (auto f : {decode_mma_kernel<kFp16, D, G, false>, decode_mma_kernel<kFp16, D, G, true>}) {
+      const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, MmaCfg<D>::kSmemBytes);
+      if (e != cudaSuccess) return static_cast<int>(e);
+    }
+    return 0;
   });
   if (ce != 0) return ce;
   kern<<<dim3(p.Hkv * (p.group / G), a.S, a.B), kMmaThreads, MmaCfg<D>::kSmemBytes, stream>>>(mk, mv, p);

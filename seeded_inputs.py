@@ -47,6 +47,9 @@ CONFIGS = {
     # the same bytes), with its own queries; splits are per key shard
     "decode_long": dict(B=4, Nk=131072, H=32, D=128, dtype="bf16", scale=1.0 / math.sqrt(128),
                         num_splits=64, seed=7, cache_of="decode"),
+    # the grouped decode workload with its cache in a paged pool: pages of 16 rows at positions of
+    # a seeded permutation of the pool, one block-table row per sequence
+    "decode_paged": dict(page_size=16, seed=8, cache_of="decode_gqa"),
 }
 
 
