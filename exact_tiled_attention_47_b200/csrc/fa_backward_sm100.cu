@@ -43,9 +43,25 @@ namespace {
 
 constexpr int kBT = 128;  // rows per tile (queries or keys)
 constexpr int kHalf = 64;  // columns of a half block
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+// Column groups per half block: the half's 64 columns are split between kCG warps on each quarter of
+// the TMEM lanes (the elementwise work needs no exchange between them: P comes from the stored LSE).
+// Two groups (16 compute warps, 88-92 registers) gave the same gradients bit for bit but were 3-4 %
+// slower than one at both head dims, so one is the default.
+#ifndef FA_BWD_CG
+#define FA_BWD_CG 1
+#endif
+constexpr int kCG = FA_BWD_CG;
+static_assert(kCG == 1 || kCG == 2 || kCG == 4, "column groups: 1, 2 or 4");
+constexpr int kChunksPerGroup = 4 / kCG;  // 16-column chunks per warp and block half
+constexpr int kComputeWarps = 8 * kCG;
+constexpr int kThreads = (kComputeWarps + 2) * 32;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kMmaWarp = kComputeWarps + 1;
+// Where chunk c (16 columns) of a half keeps its packed 16-bit P or dS: inside the columns its own
+// column group has already read, so no group overwrites values another group has yet to load.
+__host__ __device__ constexpr uint32_t packed_col(int c) {
+  return static_cast<uint32_t>(16 * kChunksPerGroup * (c / kChunksPerGroup) + 8 * (c % kChunksPerGroup));
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr int kMaxStages = 3;  // streamed-tile stages: 3 at D = 64, 2 at D = 128 (shared memory)
@@ -224,12 +240,13 @@ __device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint32_t a, uint32_t b, 
   }
 }
 
-// d += A (TMEM, 128 x 64 packed 16-bit) * B (shared, N-major, the 64 rows of a half block from b)
+// d += A (TMEM, 128 x 64 packed 16-bit, chunk kk at packed_col(kk)) * B (shared, N-major, the 64
+// rows of a half block from b)
 __device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, uint32_t idesc,
                                             bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < kHalf / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, kPanelBytes, 1024), idesc,
+    mma_ts(d_tmem, a_tmem + packed_col(kk), smem_desc_sw128(b + kk * 2048, kPanelBytes, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -276,7 +293,7 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
     }
     for (int hh = 0; hh < 2; ++hh) {
       mbar_init(&bars->s_full[hh], 1);
-      mbar_init(&bars->p_full[hh], 4);
+      mbar_init(&bars->p_full[hh], 4 * kCG);
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
@@ -415,7 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int hh = warp >> 2;  // half of every key block this warp works on
+    const int hh = warp / (4 * kCG);          // half of every key block this warp works on
+    const int cg = (warp >> 2) % kCG;          // its column group within the half
+    const int c_lo = cg * kChunksPerGroup;     // first 16-column chunk of the group
     const int r = (warp & 3) * 32 + lane;
     const int qi = m0 + r;
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -437,16 +456,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool masked = (j + 1) * kBT > tile_lim;
       const int lim = row_lim - j * kBT;
-      // the half's 64 key columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      // the group's key columns of the half in 16-column chunks; chunk c+1 is loaded while chunk c is
+      // computed
       const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
       uint32_t sb[2][16], db[2][16];
-      tmem_ld16_async(cs, sb[0]);
-      tmem_ld16_async(cd, db[0]);
+      tmem_ld16_async(cs + 16 * c_lo, sb[0]);
+      tmem_ld16_async(cd + 16 * c_lo, db[0]);
       tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int cur = c & 1;
-        if (c + 1 < 4) {
+      for (int ci = 0; ci < kChunksPerGroup; ++ci) {
+        const int c = c_lo + ci, cur = ci & 1;
+        if (ci + 1 < kChunksPerGroup) {
           tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
           tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
         }
@@ -462,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           pk[i] = pack2<kFp16>(p0 * (__uint_as_float(db[cur][2 * i]) - dr), p1 * (__uint_as_float(db[cur][2 * i + 1]) - dr));
         }
-        tmem_st8(cd + 8 * c, pk);  // dS over the half's dP columns already read
-        if (c + 1 < 4) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+        tmem_st8(cd + packed_col(c), pk);  // dS over dP columns this group has already read
+        if (ci + 1 < kChunksPerGroup) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -474,9 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const size_t row = static_cast<size_t>(u.q_row0 + min(qi, Lq - 1)) * p.H + h;
-      // the two halves of warps store the two halves of the row
+      // the 2 kCG groups of warps on this lane quarter store their shares of the row's 32-column chunks
+      const int gi = hh * kCG + cg;
       store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, p.status, p.g0_n,
-                                        hh * D / 64, (hh + 1) * D / 64);
+                                        gi * (D / 32) / (2 * kCG), (gi + 1) * (D / 32) / (2 * kCG));
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -632,7 +653,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int hh = warp >> 2;  // half of every query block this warp works on
+    const int hh = warp / (4 * kCG);          // half of every query block this warp works on
+    const int cg = (warp >> 2) % kCG;          // its column group within the half
+    const int c_lo = cg * kChunksPerGroup;     // first 16-column chunk of the group
     const int r = (warp & 3) * 32 + lane;
     const int kj = n0 + r;  // this thread's key
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -650,16 +673,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // have P = 0 through their +inf LSE
       const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
       const int q_lo = (kj < p.prefix) ? -kBT : kj - diag - i * kBT;  // columns c < q_lo are masked
-      // the half's 64 query columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      // the group's query columns of the half in 16-column chunks; chunk c+1 is loaded while chunk c
+      // is computed
       const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
       uint32_t sb[2][16], db[2][16];
-      tmem_ld16_async(cs, sb[0]);
-      tmem_ld16_async(cd, db[0]);
+      tmem_ld16_async(cs + 16 * c_lo, sb[0]);
+      tmem_ld16_async(cd + 16 * c_lo, db[0]);
       tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int cur = c & 1;
-        if (c + 1 < 4) {
+      for (int ci = 0; ci < kChunksPerGroup; ++ci) {
+        const int c = c_lo + ci, cur = ci & 1;
+        if (ci + 1 < kChunksPerGroup) {
           tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
           tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
         }
@@ -683,9 +707,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           dk[2 * q4] = pack2<kFp16>(dsv[0], dsv[1]);
           dk[2 * q4 + 1] = pack2<kFp16>(dsv[2], dsv[3]);
         }
-        tmem_st8(cs + 8 * c, pk);  // P^T over the half's S^T columns already read
-        tmem_st8(cd + 8 * c, dk);  // dS^T over the half's dP^T columns already read
-        if (c + 1 < 4) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+        tmem_st8(cs + packed_col(c), pk);  // P^T over S^T columns this group has already read
+        tmem_st8(cd + packed_col(c), dk);  // dS^T over dP^T columns this group has already read
+        if (ci + 1 < kChunksPerGroup) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -696,8 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const size_t row = (static_cast<size_t>(u.k_row0 + min(kj, Lk - 1)) * p.H + h) * D;
-      if (hh == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk, p.status, p.g1_n);  // dV
-      else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk, p.status, p.g0_n);  // dK
+      // warps of half 0 store dV, those of half 1 dK, each column group its share of the 32-column chunks
+      const int ch_lo = cg * (D / 32) / kCG, ch_hi = (cg + 1) * (D / 32) / kCG;
+      if (hh == 0)
+        store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk, p.status, p.g1_n, ch_lo, ch_hi);
+      else
+        store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk, p.status, p.g0_n, ch_lo,
+                                          ch_hi);
     }
   }
   bwd_teardown(bars, warp, tbase);
