@@ -222,32 +222,49 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 
-__device__ __forceinline__ void smem_desc_pair_k(uint32_t a, uint32_t b, int kk, uint64_t& da, uint64_t& db) {
-  // K-major, 128B swizzle: 16-element K steps advance 32 bytes inside a 128-byte row; every 4 steps
-  // move to the next 64-column panel.  SBO = 8 rows * 128 B.
-  const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-  da = smem_desc_sw128(a + off, 16, 1024);
-  db = smem_desc_sw128(b + off, 16, 1024);
+// The MMA thread issues every product of the CTA, and at N = 64 an MMA takes about 64 cycles of
+// issue (twice its tensor work), so the per-MMA instruction count matters: every shared-memory
+// descriptor is derived from one built once per tile buffer by adding a constant offset (its start
+// address field, bits 0-13 in 16-byte units, cannot carry: shared memory ends below 2^18 bytes).
+__device__ __forceinline__ uint64_t desc_kmajor(const void* tile) { return smem_desc_sw128(smem_addr(tile), 16, 1024); }
+__device__ __forceinline__ uint64_t desc_nmajor(const void* tile) {
+  return smem_desc_sw128(smem_addr(tile), kPanelBytes, 1024);
+}
+// offset (16-byte units) of K step kk in a K-major tile: 16-element steps advance 32 bytes inside a
+// 128-byte row; every 4 steps move to the next 64-column panel
+__host__ __device__ constexpr uint32_t kstep_off(int kk) {
+  return static_cast<uint32_t>(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
 }
 
+// Two independent products d0 = a0 b0^T and d1 = a1 b1^T (both operands K-major in shared memory,
+// K = D) with their K steps interleaved.
 template <int D>
-__device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint32_t a, uint32_t b, uint32_t idesc) {
+__device__ __forceinline__ void mma_kk2(uint32_t d0, uint64_t a0, uint64_t b0, uint32_t d1, uint64_t a1, uint64_t b1,
+                                        uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    uint64_t da, db;
-    smem_desc_pair_k(a, b, kk, da, db);
-    mma_ss(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+    mma_ss(d0, a0 + kstep_off(kk), b0 + kstep_off(kk), idesc, kk > 0 ? 1u : 0u);
+    mma_ss(d1, a1 + kstep_off(kk), b1 + kstep_off(kk), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// d += A (TMEM, 128 x 64 packed 16-bit, chunk kk at packed_col(kk)) * B (shared, N-major, the 64
-// rows of a half block from b)
-__device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, uint32_t idesc,
+// d += A (TMEM, 128 x 64 packed 16-bit, chunk kk at packed_col(kk)) * B (shared, N-major: the 64 rows
+// of a half block, b the descriptor of its first row); 16 rows = two 8-row swizzle atoms = 2048 bytes
+__device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                             bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < kHalf / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + packed_col(kk), smem_desc_sw128(b + kk * 2048, kPanelBytes, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d_tmem, a_tmem + packed_col(kk), b + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Two independent TS products with their K steps interleaved.
+__device__ __forceinline__ void mma_tn_half2(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t d1, uint32_t a1,
+                                             uint64_t b1, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kHalf / 16; ++kk) {
+    mma_ts(d0, a0 + packed_col(kk), b0 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d1, a1 + packed_col(kk), b1 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 // Byte offset of row 64 in a 128-row swizzled tile (rows are 128 bytes in every 64-column panel).
@@ -396,10 +413,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int fmt = kFp16 ? 0 : 1;
       constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      const uint64_t d_q = desc_kmajor(sQ), d_do = desc_kmajor(sDO);
+      const uint64_t d_k = desc_kmajor(sK(0)), d_v = desc_kmajor(sV(0)), d_kn = desc_nmajor(sK(0));
+      // offset (16-byte units) of half hh of stage st's tile from stage 0's
+      auto half_off = [&](int st, int hh) { return static_cast<uint64_t>((st * C::kTileBytes + kHalfRowOff * hh) >> 4); };
       // S = Q K_j^T and dP = dO V_j^T of half hh (keys 64 hh .. 64 hh + 63 of block j)
       auto issue_s = [&](int st, int hh) {
-        mma_kk<D>(tbase + kColS + kHalf * hh, smem_addr(sQ), smem_addr(sK(st)) + kHalfRowOff * hh, idesc_s);
-        mma_kk<D>(tbase + kColDP + kHalf * hh, smem_addr(sDO), smem_addr(sV(st)) + kHalfRowOff * hh, idesc_s);
+        mma_kk2<D>(tbase + kColS + kHalf * hh, d_q, d_k + half_off(st, hh), tbase + kColDP + kHalf * hh, d_do,
+                   d_v + half_off(st, hh), idesc_s);
         mma_commit(&bars->s_full[hh]);
       };
       bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
@@ -415,8 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&bars->p_full[hh], j & 1, abort_flag, p.status))) break;
           tc_fence_after();
           // dQ += dS_hh K_j[hh]
-          mma_tn_half(tbase + kColA, tbase + kColDP + kHalf * hh, smem_addr(sK(st)) + kHalfRowOff * hh, idesc_g,
-                      j > 0 || hh > 0);
+          mma_tn_half(tbase + kColA, tbase + kColDP + kHalf * hh, d_kn + half_off(st, hh), idesc_g, j > 0 || hh > 0);
           if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
           if (j + 1 < n) {
             const int st1 = (j + 1) % C::kSt;
@@ -615,10 +635,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int fmt = kFp16 ? 0 : 1;
       constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      const uint64_t d_k = desc_kmajor(sK), d_v = desc_kmajor(sV);
+      const uint64_t d_q = desc_kmajor(sQ(0)), d_do = desc_kmajor(sDO(0));
+      const uint64_t d_qn = desc_nmajor(sQ(0)), d_don = desc_nmajor(sDO(0));
+      // offset (16-byte units) of half hh of stage st's tile from stage 0's
+      auto half_off = [&](int st, int hh) { return static_cast<uint64_t>((st * C::kTileBytes + kHalfRowOff * hh) >> 4); };
       // S^T = K Q_i^T and dP^T = V dO_i^T of half hh (queries 64 hh .. 64 hh + 63 of block i)
       auto issue_s = [&](int st, int hh) {
-        mma_kk<D>(tbase + kColS + kHalf * hh, smem_addr(sK), smem_addr(sQ(st)) + kHalfRowOff * hh, idesc_s);
-        mma_kk<D>(tbase + kColDP + kHalf * hh, smem_addr(sV), smem_addr(sDO(st)) + kHalfRowOff * hh, idesc_s);
+        mma_kk2<D>(tbase + kColS + kHalf * hh, d_k, d_q + half_off(st, hh), tbase + kColDP + kHalf * hh, d_v,
+                   d_do + half_off(st, hh), idesc_s);
         mma_commit(&bars->s_full[hh]);
       };
       bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
@@ -635,9 +660,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const bool acc = jj > 0 || hh > 0;
           // dV += P^T_hh dO_i[hh],  dK += dS^T_hh Q_i[hh]
-          mma_tn_half(tbase + kColA, tbase + kColS + kHalf * hh, smem_addr(sDO(st)) + kHalfRowOff * hh, idesc_g, acc);
-          mma_tn_half(tbase + kColA + D, tbase + kColDP + kHalf * hh, smem_addr(sQ(st)) + kHalfRowOff * hh, idesc_g,
-                      acc);
+          mma_tn_half2(tbase + kColA, tbase + kColS + kHalf * hh, d_don + half_off(st, hh), tbase + kColA + D,
+                       tbase + kColDP + kHalf * hh, d_qn + half_off(st, hh), idesc_g, acc);
           if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
           if (jj + 1 < n) {
             const int st1 = (jj + 1) % C::kSt;
