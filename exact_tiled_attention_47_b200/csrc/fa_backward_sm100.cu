@@ -10,28 +10,28 @@
 // Three kernels, no atomics:
 //   bwd_rowterm_kernel  Drow[b,h,i] (fp32), one thread per (b, i, h) row.
 //   bwd_dq_kernel       CTA = one 128-row query tile.  Per key block j: S = Q K_j^T and
-//                       dP = dO V_j^T into TMEM, the four compute warps (thread = query row) form dS
-//                       32 columns at a time and write it (bf16/fp16) over the first 64 columns of
-//                       dP, then dQ += dS K_j accumulates in TMEM.  dQ * scale is written at the end.
+//                       dP = dO V_j^T into TMEM, the eight compute warps (thread = query row, two
+//                       warps per TMEM lane quarter, one per 64-column half) form dS and pack it
+//                       (bf16/fp16) over the dP columns they have read, then dQ += dS K_j accumulates
+//                       in TMEM.  dQ * scale is written at the end.
 //   bwd_dkdv_kernel     CTA = one 128-row key tile.  Per query block i: S^T = K Q_i^T and
 //                       dP^T = V dO_i^T into TMEM, the compute warps (thread = key row) form P^T and
-//                       dS^T 32 query columns at a time (the block's LSE and Drow come through shared
-//                       memory) and write them over S^T and dP^T, then dV += P^T dO_i and
-//                       dK += dS^T Q_i accumulate in TMEM.  dV and dK * scale are written at the end.
+//                       dS^T (the block's LSE and Drow come through shared memory) and pack both over
+//                       the dP^T columns they have read, then dV += P^T dO_i and dK += dS^T Q_i
+//                       accumulate in TMEM.  dV and dK * scale are written at the end.
 // Both recompute S and dP (two more GEMMs than the minimum) so that each gradient is owned by one
-// CTA and accumulates in TMEM.  Each streamed 128-row block is processed as two 64-column halves that
-// form two independent pipelines: warps 0-3 compute half 0 and warps 4-7 half 1 (the same TMEM lanes,
-// different columns), warp 8 is the TMA producer, and warp 9 owns TMEM and issues every tcgen05.mma
-// from one thread.  For each half it issues S and dP (N = 64), waits for that half's P/dS, issues the
-// half's gradient products (K = 64) and at once the next block's S and dP of the same half, so the
-// tensor core works on one half while the other half's softmax-derivative runs (the tensor core runs
-// one thread's MMAs in order, which orders each half's next S/dP after the products that read its
-// P/dS columns).  The MMA forms are those of the forward kernel: SS with both operands K-major (S, dP)
-// and TS with the A operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal runs skip
-// fully masked blocks; masking is applied on the blocks that cross the diagonal and at the sequence
-// ends.  The masks and layouts are those of the forward kernel: causal (bottom-right aligned), the
-// prefix-LM mask (keys [0, prefix) visible to every query of the sequence) and packed varlen
-// sequences indexed through cu_seqlens (LSE and Drow [H, total]).
+// CTA and accumulates in TMEM.  Warp 8 is the TMA producer; warp 9 owns TMEM and issues every
+// tcgen05.mma from one thread.  A single thread issues an MMA about every 64 cycles whatever N up
+// to 128 (measured), so S and dP are whole-block products (M = N = 128) and the schedule keeps the
+// issue thread off the compute warps' path: S is released for the next block's S as soon as the
+// compute warps hold it in registers, and dP goes into one of two TMEM buffers two blocks ahead
+// (after the gradient products that read that buffer; with one buffer, as in dK/dV at D = 128,
+// right after them).  The MMA forms are those of the forward kernel: SS with both operands K-major
+// (S, dP) and TS with the A operand in TMEM and an N-major B in shared memory (dQ, dV, dK).  Causal
+// runs skip fully masked blocks; masking is applied on the blocks that cross the diagonal and at
+// the sequence ends.  The masks and layouts are those of the forward kernel: causal (bottom-right
+// aligned), the prefix-LM mask (keys [0, prefix) visible to every query of the sequence) and packed
+// varlen sequences indexed through cu_seqlens (LSE and Drow [H, total]).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -42,41 +42,38 @@ namespace fa {
 namespace {
 
 constexpr int kBT = 128;  // rows per tile (queries or keys)
-constexpr int kHalf = 64;  // columns of a half block
-// Column groups per half block: the half's 64 columns are split between kCG warps on each quarter of
-// the TMEM lanes (the elementwise work needs no exchange between them: P comes from the stored LSE).
-// Two groups (16 compute warps, 88-92 registers) gave the same gradients bit for bit but were 3-4 %
-// slower than one at both head dims, so one is the default.
-#ifndef FA_BWD_CG
-#define FA_BWD_CG 1
-#endif
-constexpr int kCG = FA_BWD_CG;
-static_assert(kCG == 1 || kCG == 2 || kCG == 4, "column groups: 1, 2 or 4");
-constexpr int kChunksPerGroup = 4 / kCG;  // 16-column chunks per warp and block half
-constexpr int kComputeWarps = 8 * kCG;
-constexpr int kThreads = (kComputeWarps + 2) * 32;
-constexpr int kProducerWarp = kComputeWarps;
-constexpr int kMmaWarp = kComputeWarps + 1;
-// Where chunk c (16 columns) of a half keeps its packed 16-bit P or dS: inside the columns its own
-// column group has already read, so no group overwrites values another group has yet to load.
-__host__ __device__ constexpr uint32_t packed_col(int c) {
-  return static_cast<uint32_t>(16 * kChunksPerGroup * (c / kChunksPerGroup) + 8 * (c % kChunksPerGroup));
-}
+constexpr int kThreads = 320;  // 8 compute warps, a TMA producer warp, an MMA warp
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr int kMaxStages = 3;  // streamed-tile stages: 3 at D = 64, 2 at D = 128 (shared memory)
-constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256;  // S (P over it), dP (dS over it), accumulators
+// Tensor memory: S (or S^T) in columns [0, 128), one or two dP (dP^T) buffers of 128 columns after it
+// (the compute warps pack their 16-bit results into the dP columns they have read), then the
+// accumulators (dQ; or dV and dK).
+constexpr uint32_t kColS = 0, kColDP = 128;
 
 template <int D>
 struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kTileBytes = kBT * D * 2;
   static constexpr int kSt = (D == 64) ? 3 : 2;
+  // dP buffers: two where they fit next to the accumulators (dQ: always; dK/dV: D = 64)
+  template <bool kDkdv>
+  static constexpr int kDPBufs = (!kDkdv || D == 64) ? 2 : 1;
+  template <bool kDkdv>
+  static constexpr uint32_t kColAcc = kColDP + 128 * kDPBufs<kDkdv>;
   static constexpr int kUsed = (2 + 2 * kSt) * kTileBytes + 2 * kSt * kBT * 4 + 256 + 1024;
   // at least 120 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
   static constexpr int kSmemBytes = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  // dQ kernel: K and V stream through rings of their own, K three deep (S(j+1) is issued while
+  // dQ(j) may still read K(j)), V three deep at D = 64 and two at D = 128, where shared memory ends
+  // (V is read only by dP, which runs two blocks ahead; two V slots measured 2.6 % slower at D = 64)
+  static constexpr int kKSt = 3, kVSt = (D == 64) ? 3 : 2;
+  static constexpr int kDqUsed = (2 + kKSt + kVSt) * kTileBytes + 256 + 1024;
+  static constexpr int kDqSmemBytes = kDqUsed > 120 * 1024 ? kDqUsed : 120 * 1024;
 };
-static_assert(BwdCfg<128>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(BwdCfg<128>::kSmemBytes <= 232448 && BwdCfg<128>::kDqSmemBytes <= 232448, "shared memory budget");
 
 struct BwdParams {
   const float* lse;   // [B, H, Nq]
@@ -154,7 +151,10 @@ struct BwdBars {
   uint64_t fixed_full;                           // the CTA's own tiles (Q + dO, or K + V)
   uint64_t st_full[kMaxStages], st_empty[kMaxStages];  // streamed tiles (K + V, or Q + dO)
   uint64_t stat_full[kMaxStages];                      // dK/dV: the streamed block's LSE and Drow in shared memory
-  uint64_t s_full[2], p_full[2];                 // per half block
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];  // dQ: the K and V rings
+  uint64_t s_full;   // S and dP of the next block are in TMEM (one phase per block)
+  uint64_t s_read;   // the compute warps hold the block's S in registers: S may be overwritten
+  uint64_t p_full;   // the block's packed dS (and P^T) are in TMEM
   uint64_t o_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -236,39 +236,40 @@ __host__ __device__ constexpr uint32_t kstep_off(int kk) {
   return static_cast<uint32_t>(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
 }
 
-// Two independent products d0 = a0 b0^T and d1 = a1 b1^T (both operands K-major in shared memory,
-// K = D) with their K steps interleaved.
+// d = a b^T over K = D (both operands K-major in shared memory; a and b are descriptors)
 template <int D>
-__device__ __forceinline__ void mma_kk2(uint32_t d0, uint64_t a0, uint64_t b0, uint32_t d1, uint64_t a1, uint64_t b1,
-                                        uint32_t idesc) {
+__device__ __forceinline__ void mma_kk(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    mma_ss(d0, a0 + kstep_off(kk), b0 + kstep_off(kk), idesc, kk > 0 ? 1u : 0u);
-    mma_ss(d1, a1 + kstep_off(kk), b1 + kstep_off(kk), idesc, kk > 0 ? 1u : 0u);
+  for (int kk = 0; kk < D / 16; ++kk) mma_ss(d, a + kstep_off(kk), b + kstep_off(kk), idesc, kk > 0 ? 1u : 0u);
+}
+
+// Where 16-column chunk kk (0..7) of a block keeps its packed 16-bit values in the dP buffer: the
+// compute warps of column half c = kk / 4 write chunk ci = kk % 4 over the dP columns they have just
+// read.  dQ kernel: dS at 64 c + 8 ci.  dK/dV kernel: dS^T at 64 c + 16 ci and P^T 8 columns after it.
+__host__ __device__ constexpr uint32_t ds_col_dq(int kk) { return static_cast<uint32_t>(64 * (kk >> 2) + 8 * (kk & 3)); }
+__host__ __device__ constexpr uint32_t ds_col_dkdv(int kk) {
+  return static_cast<uint32_t>(64 * (kk >> 2) + 16 * (kk & 3));
+}
+
+// d (+)= A (TMEM, 128 x 128 packed 16-bit, chunk kk at a_tmem + col(kk)) * B (shared, N-major 128
+// rows from the descriptor b; 16 rows = two 8-row swizzle atoms = 2048 bytes).  Two products
+// (d0, d1) have their K steps interleaved.
+template <uint32_t (*col)(int)>
+__device__ __forceinline__ void mma_tn(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kBT / 16; ++kk)
+    mma_ts(d, a + col(kk), b + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+template <uint32_t (*col)(int)>
+__device__ __forceinline__ void mma_tn2(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t d1, uint32_t a1, uint64_t b1,
+                                        uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kBT / 16; ++kk) {
+    mma_ts(d0, a0 + col(kk), b0 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d1, a1 + col(kk), b1 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
-// d += A (TMEM, 128 x 64 packed 16-bit, chunk kk at packed_col(kk)) * B (shared, N-major: the 64 rows
-// of a half block, b the descriptor of its first row); 16 rows = two 8-row swizzle atoms = 2048 bytes
-__device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                            bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < kHalf / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + packed_col(kk), b + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// Two independent TS products with their K steps interleaved.
-__device__ __forceinline__ void mma_tn_half2(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t d1, uint32_t a1,
-                                             uint64_t b1, uint32_t idesc, bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < kHalf / 16; ++kk) {
-    mma_ts(d0, a0 + packed_col(kk), b0 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
-    mma_ts(d1, a1 + packed_col(kk), b1 + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
-// Byte offset of row 64 in a 128-row swizzled tile (rows are 128 bytes in every 64-column panel).
-constexpr uint32_t kHalfRowOff = kHalf * 128;
 
 // Every lane of the warp loads (tcgen05.ld is warp-collective); only lanes with store write the row.
 // Columns [32 * ch_lo, 32 * ch_hi) of the row.
@@ -308,10 +309,17 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
       mbar_init(&bars->st_empty[s], 1);
       mbar_init(&bars->stat_full[s], 1);
     }
-    for (int hh = 0; hh < 2; ++hh) {
-      mbar_init(&bars->s_full[hh], 1);
-      mbar_init(&bars->p_full[hh], 4 * kCG);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
     }
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_read, 8);
+    mbar_init(&bars->p_full, 8);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -349,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sDO = smem + C::kTileBytes;
-  auto sK = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
-  auto sV = [&](int st) { return smem + (2 + C::kSt + st) * C::kTileBytes; };
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
+  auto sK = [&](int ks) { return smem + (2 + ks) * C::kTileBytes; };
+  auto sV = [&](int vs) { return smem + (2 + C::kKSt + vs) * C::kTileBytes; };
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + C::kKSt + C::kVSt) * C::kTileBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const BwdUnit u = bwd_unit<true>(p, warp, lane, &bars->unit_b, &bars->unit_t);
@@ -390,61 +398,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(&tm_q, &bars->fixed_full, sQ + pn * kPanelBytes, pn * 64, h, u.q_row0 + m0);
         tma_load_3d(&tm_do, &bars->fixed_full, sDO + pn * kPanelBytes, pn * 64, h, u.q_row0 + m0);
       }
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        const int st = j % C::kSt;
-        if (!(ok = mbar_wait(&bars->st_empty[st], ((j / C::kSt) & 1) ^ 1, abort_flag, p.status))) break;
-        mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::kTileBytes);
+        const int ks = j % C::kKSt, vs = j % C::kVSt;
+        if (!(ok = mbar_wait(&bars->k_empty[ks], ((j / C::kKSt) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&bars->k_full[ks], C::kTileBytes);
 #pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d_hint(&tm_k, &bars->st_full[st], sK(st) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
-          tma_load_3d_hint(&tm_v, &bars->st_full[st], sV(st) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
-        }
-        issued = j + 1;
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(&tm_k, &bars->k_full[ks], sK(ks) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
+        k_issued = j + 1;
+        if (!(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVSt) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(&tm_v, &bars->v_full[vs], sV(vs) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
+        v_issued = j + 1;
       }
-      if (!ok) {
+      if (!ok) {  // the newest copy into each slot is the only one that can still be in flight
         drain_wait(&bars->fixed_full, 0);
-        for (int j = max(0, issued - C::kSt); j < issued; ++j) drain_wait(&bars->st_full[j % C::kSt], (j / C::kSt) & 1);
+        for (int j = max(0, k_issued - C::kKSt); j < k_issued; ++j) drain_wait(&bars->k_full[j % C::kKSt], (j / C::kKSt) & 1);
+        for (int j = max(0, v_issued - C::kVSt); j < v_issued; ++j) drain_wait(&bars->v_full[j % C::kVSt], (j / C::kVSt) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
+      // Block j: S = Q K_j^T into the S columns and dP = dO V_j^T into dP buffer j % 2 (N = 128, so
+      // each MMA carries twice the work of a half block at the same issue cost), then, once the
+      // compute warps have packed dS into that buffer, dQ += dS K_j.  S(j+1) is issued as soon as the
+      // compute warps hold S(j) in registers; dP(j+2) goes into buffer j % 2 right after dQ(j), so
+      // only S is issued between the blocks of the compute warps.
       constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      constexpr uint32_t col_acc = C::template kColAcc<false>;
       const uint64_t d_q = desc_kmajor(sQ), d_do = desc_kmajor(sDO);
       const uint64_t d_k = desc_kmajor(sK(0)), d_v = desc_kmajor(sV(0)), d_kn = desc_nmajor(sK(0));
-      // offset (16-byte units) of half hh of stage st's tile from stage 0's
-      auto half_off = [&](int st, int hh) { return static_cast<uint64_t>((st * C::kTileBytes + kHalfRowOff * hh) >> 4); };
-      // S = Q K_j^T and dP = dO V_j^T of half hh (keys 64 hh .. 64 hh + 63 of block j)
-      auto issue_s = [&](int st, int hh) {
-        mma_kk2<D>(tbase + kColS + kHalf * hh, d_q, d_k + half_off(st, hh), tbase + kColDP + kHalf * hh, d_do,
-                   d_v + half_off(st, hh), idesc_s);
-        mma_commit(&bars->s_full[hh]);
+      auto slot_off = [&](int slot) { return static_cast<uint64_t>((slot * C::kTileBytes) >> 4); };
+      auto wait_k = [&](int jb) {
+        return mbar_wait(&bars->k_full[jb % C::kKSt], (jb / C::kKSt) & 1, abort_flag, p.status);
       };
-      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
-                mbar_wait(&bars->st_full[0], 0, abort_flag, p.status);
+      auto wait_v = [&](int jb) {
+        return mbar_wait(&bars->v_full[jb % C::kVSt], (jb / C::kVSt) & 1, abort_flag, p.status);
+      };
+      auto issue_S = [&](int jb) { mma_kk<D>(tbase + kColS, d_q, d_k + slot_off(jb % C::kKSt), idesc_s); };
+      auto issue_dP = [&](int jb) {  // V(jb) is released once this product has completed
+        mma_kk<D>(tbase + kColDP + 128 * (jb & 1), d_do, d_v + slot_off(jb % C::kVSt), idesc_s);
+        mma_commit(&bars->v_empty[jb % C::kVSt]);
+      };
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(0, 1);
+        issue_S(0);
+        issue_dP(0);
+        mma_commit(&bars->s_full);
+        if (n > 1 && (ok = wait_v(1))) {
+          tc_fence_after();
+          issue_dP(1);
+        }
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j % C::kSt;
-        for (int hh = 0; hh < 2; ++hh) {
-          if (!(ok = mbar_wait(&bars->p_full[hh], j & 1, abort_flag, p.status))) break;
+        if (j + 1 < n) {
+          // the compute warps have S(j) in registers: S(j+1) may overwrite it
+          if (!(ok = mbar_wait(&bars->s_read, j & 1, abort_flag, p.status) && wait_k(j + 1))) break;
           tc_fence_after();
-          // dQ += dS_hh K_j[hh]
-          mma_tn_half(tbase + kColA, tbase + kColDP + kHalf * hh, d_kn + half_off(st, hh), idesc_g, j > 0 || hh > 0);
-          if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
-          if (j + 1 < n) {
-            const int st1 = (j + 1) % C::kSt;
-            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((j + 1) / C::kSt) & 1, abort_flag, p.status)))
-              break;
-            tc_fence_after();
-            issue_s(st1, hh);
-          }
+          issue_S(j + 1);
+          mma_commit(&bars->s_full);  // S(j+1) and dP(j+1)
+        }
+        if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_tn<ds_col_dq>(tbase + col_acc, tbase + kColDP + 128 * (j & 1), d_kn + slot_off(j % C::kKSt), idesc_g,
+                          j > 0);
+        mma_commit(&bars->k_empty[j % C::kKSt]);  // K(j): S(j) and dQ(j) issued
+        if (j + 2 < n) {
+          if (!(ok = wait_v(j + 2))) break;
+          tc_fence_after();
+          issue_dP(j + 2);  // into buffer j % 2, after dQ(j) (the tensor core keeps one thread's order)
         }
       }
       if (ok) mma_commit(&bars->o_done);
@@ -452,9 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int hh = warp / (4 * kCG);          // half of every key block this warp works on
-    const int cg = (warp >> 2) % kCG;          // its column group within the half
-    const int c_lo = cg * kChunksPerGroup;     // first 16-column chunk of the group
+    const int hc = warp >> 2;  // column half of every key block this warp works on
     const int r = (warp & 3) * 32 + lane;
     const int qi = m0 + r;
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -472,28 +499,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      if (!(ok = warp_wait(&bars->s_full[hh], j & 1, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(&bars->s_full, j & 1, abort_flag, p.status))) break;
       tc_fence_after();
       const bool masked = (j + 1) * kBT > tile_lim;
       const int lim = row_lim - j * kBT;
-      // the group's key columns of the half in 16-column chunks; chunk c+1 is loaded while chunk c is
-      // computed
-      const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
+      // the half's 64 key columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      const uint32_t cs = lane_base + kColS + 64 * hc, cd = lane_base + kColDP + 128 * (j & 1) + 64 * hc;
       uint32_t sb[2][16], db[2][16];
-      tmem_ld16_async(cs + 16 * c_lo, sb[0]);
-      tmem_ld16_async(cd + 16 * c_lo, db[0]);
+      tmem_ld16_async(cs, sb[0]);
+      tmem_ld16_async(cd, db[0]);
       tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int ci = 0; ci < kChunksPerGroup; ++ci) {
-        const int c = c_lo + ci, cur = ci & 1;
-        if (ci + 1 < kChunksPerGroup) {
+      for (int c = 0; c < 4; ++c) {
+        const int cur = c & 1;
+        if (c + 1 < 4) {
           tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
           tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
         }
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int c0 = kHalf * hh + 16 * c + 2 * i;  // key column in the block
+          const int c0 = 64 * hc + 16 * c + 2 * i;  // key column in the block
           float p0 = ex2(fmaf(__uint_as_float(sb[cur][2 * i]), sl2, -lse2));
           float p1 = ex2(fmaf(__uint_as_float(sb[cur][2 * i + 1]), sl2, -lse2));
           if (masked) {
@@ -502,22 +528,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           pk[i] = pack2<kFp16>(p0 * (__uint_as_float(db[cur][2 * i]) - dr), p1 * (__uint_as_float(db[cur][2 * i + 1]) - dr));
         }
-        tmem_st8(cd + packed_col(c), pk);  // dS over dP columns this group has already read
-        if (ci + 1 < kChunksPerGroup) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+        tmem_st8(cd + 8 * c, pk);  // dS over dP columns this warp has already read (ds_col_dq)
+        if (c + 1 < 4) {
+          tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+          if (c == 2) {  // all of this warp's S columns are in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->s_read);
+          }
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[hh]);
+      if (lane == 0) mbar_arrive(&bars->p_full);
     }
     if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       const size_t row = static_cast<size_t>(u.q_row0 + min(qi, Lq - 1)) * p.H + h;
-      // the 2 kCG groups of warps on this lane quarter store their shares of the row's 32-column chunks
-      const int gi = hh * kCG + cg;
-      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + kColA, p.scale, qi < Lq, p.status, p.g0_n,
-                                        gi * (D / 32) / (2 * kCG), (gi + 1) * (D / 32) / (2 * kCG));
+      // the two column halves of warps store the two halves of the row
+      store_grad_row<D, kFp16, kOutF32>(p.g0, row * D, lane_base + C::template kColAcc<false>, p.scale, qi < Lq,
+                                        p.status, p.g0_n, hc * D / 64, (hc + 1) * D / 64);
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -632,44 +664,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
+      // Query block i (jj-th of the tile): S^T = K Q_i^T into the S columns and dP^T = V dO_i^T into a
+      // dP buffer (N = 128); once the compute warps have packed dS^T and P^T into that buffer,
+      // dV += P^T dO_i and dK += dS^T Q_i.  S^T(jj+1) is issued as soon as the compute warps hold
+      // S^T(jj) in registers.  With two dP buffers (D = 64) dP^T(jj+2) follows the products of block
+      // jj; with one (D = 128) dP^T(jj+1) does.
       constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kHalf, fmt, 0);
+      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
       constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+      constexpr int kBufs = C::template kDPBufs<true>;
+      constexpr uint32_t col_acc = C::template kColAcc<true>;
       const uint64_t d_k = desc_kmajor(sK), d_v = desc_kmajor(sV);
       const uint64_t d_q = desc_kmajor(sQ(0)), d_do = desc_kmajor(sDO(0));
       const uint64_t d_qn = desc_nmajor(sQ(0)), d_don = desc_nmajor(sDO(0));
-      // offset (16-byte units) of half hh of stage st's tile from stage 0's
-      auto half_off = [&](int st, int hh) { return static_cast<uint64_t>((st * C::kTileBytes + kHalfRowOff * hh) >> 4); };
-      // S^T = K Q_i^T and dP^T = V dO_i^T of half hh (queries 64 hh .. 64 hh + 63 of block i)
-      auto issue_s = [&](int st, int hh) {
-        mma_kk2<D>(tbase + kColS + kHalf * hh, d_k, d_q + half_off(st, hh), tbase + kColDP + kHalf * hh, d_v,
-                   d_do + half_off(st, hh), idesc_s);
-        mma_commit(&bars->s_full[hh]);
+      auto stage_off = [&](int st) { return static_cast<uint64_t>((st * C::kTileBytes) >> 4); };
+      auto wait_stage = [&](int jb) {
+        return mbar_wait(&bars->st_full[jb % C::kSt], (jb / C::kSt) & 1, abort_flag, p.status);
       };
-      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) &&
-                mbar_wait(&bars->st_full[0], 0, abort_flag, p.status);
+      auto buf = [&](int jb) { return kColDP + 128 * (jb % kBufs); };
+      auto issue_S = [&](int jb) { mma_kk<D>(tbase + kColS, d_k, d_q + stage_off(jb % C::kSt), idesc_s); };
+      auto issue_dP = [&](int jb) { mma_kk<D>(tbase + buf(jb), d_v, d_do + stage_off(jb % C::kSt), idesc_s); };
+      // dP^T of block jb + kBufs goes out after block jb's products: it needs block jb + kBufs's stage
+      // (kSt >= kBufs + 1 stages, so it is not block jb's own)
+      static_assert(C::kSt >= kBufs + 1, "stages for the dP lookahead");
+      bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) && wait_stage(0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(0, 1);
+        issue_S(0);
+        issue_dP(0);
+        mma_commit(&bars->s_full);
+        for (int jb = 1; ok && jb < kBufs && jb < n; ++jb) {  // the other buffers' first blocks
+          if ((ok = wait_stage(jb))) {
+            tc_fence_after();
+            issue_dP(jb);
+          }
+        }
       }
       for (int jj = 0; ok && jj < n; ++jj) {
         const int st = jj % C::kSt;
-        for (int hh = 0; hh < 2; ++hh) {
-          if (!(ok = mbar_wait(&bars->p_full[hh], jj & 1, abort_flag, p.status))) break;
+        if (jj + 1 < n) {
+          // the compute warps have S^T(jj) in registers: S^T(jj+1) may overwrite it (with two buffers
+          // its stage was waited for when dP^T(jj+1) was issued)
+          if (!(ok = mbar_wait(&bars->s_read, jj & 1, abort_flag, p.status))) break;
+          if (kBufs == 1 && !(ok = wait_stage(jj + 1))) break;
           tc_fence_after();
-          const bool acc = jj > 0 || hh > 0;
-          // dV += P^T_hh dO_i[hh],  dK += dS^T_hh Q_i[hh]
-          mma_tn_half2(tbase + kColA, tbase + kColS + kHalf * hh, d_don + half_off(st, hh), tbase + kColA + D,
-                       tbase + kColDP + kHalf * hh, d_qn + half_off(st, hh), idesc_g, acc);
-          if (hh == 1) mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
-          if (jj + 1 < n) {
-            const int st1 = (jj + 1) % C::kSt;
-            if (hh == 0 && !(ok = mbar_wait(&bars->st_full[st1], ((jj + 1) / C::kSt) & 1, abort_flag, p.status)))
-              break;
-            tc_fence_after();
-            issue_s(st1, hh);
-          }
+          issue_S(jj + 1);
+          if (kBufs > 1) mma_commit(&bars->s_full);  // S^T(jj+1) and dP^T(jj+1)
+        }
+        if (!(ok = mbar_wait(&bars->p_full, jj & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        // dV += P^T dO_i,  dK += dS^T Q_i  (P^T 8 columns after dS^T in every chunk)
+        mma_tn2<ds_col_dkdv>(tbase + col_acc, tbase + buf(jj) + 8, d_don + stage_off(st), tbase + col_acc + D,
+                             tbase + buf(jj), d_qn + stage_off(st), idesc_g, jj > 0);
+        mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
+        if (jj + kBufs < n) {
+          if (!(ok = wait_stage(jj + kBufs))) break;
+          tc_fence_after();
+          issue_dP(jj + kBufs);  // into block jj's buffer, after its products (the tensor core keeps order)
+          if (kBufs == 1) mma_commit(&bars->s_full);  // S^T(jj+1) and dP^T(jj+1)
         }
       }
       if (ok) mma_commit(&bars->o_done);
@@ -677,9 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bars->drain, 0);
     }
   } else {
-    const int hh = warp / (4 * kCG);          // half of every query block this warp works on
-    const int cg = (warp >> 2) % kCG;          // its column group within the half
-    const int c_lo = cg * kChunksPerGroup;     // first 16-column chunk of the group
+    constexpr int kBufs = C::template kDPBufs<true>;
+    const int hc = warp >> 2;  // column half of every query block this warp works on
     const int r = (warp & 3) * 32 + lane;
     const int kj = n0 + r;  // this thread's key
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -687,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       const int i = i_first + jj, st = jj % C::kSt;
-      if (!(ok = warp_wait(&bars->s_full[hh], jj & 1, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(&bars->s_full, jj & 1, abort_flag, p.status))) break;
       // the stage's LSE/Drow (this stage cannot be refilled before this block's P V products)
       if (!(ok = warp_wait(&bars->stat_full[st], (jj / C::kSt) & 1, abort_flag, p.status))) break;
       tc_fence_after();
@@ -697,24 +748,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // have P = 0 through their +inf LSE
       const bool masked = p.causal && (i * kBT + diag < n0 + kBT - 1);
       const int q_lo = (kj < p.prefix) ? -kBT : kj - diag - i * kBT;  // columns c < q_lo are masked
-      // the group's query columns of the half in 16-column chunks; chunk c+1 is loaded while chunk c
-      // is computed
-      const uint32_t cs = lane_base + kColS + kHalf * hh, cd = lane_base + kColDP + kHalf * hh;
+      // the half's 64 query columns in 16-column chunks; chunk c+1 is loaded while chunk c is computed
+      const uint32_t cs = lane_base + kColS + 64 * hc, cd = lane_base + kColDP + 128 * (jj % kBufs) + 64 * hc;
       uint32_t sb[2][16], db[2][16];
-      tmem_ld16_async(cs + 16 * c_lo, sb[0]);
-      tmem_ld16_async(cd + 16 * c_lo, db[0]);
+      tmem_ld16_async(cs, sb[0]);
+      tmem_ld16_async(cd, db[0]);
       tmem_wait_ld_pair(sb[0], db[0]);
 #pragma unroll
-      for (int ci = 0; ci < kChunksPerGroup; ++ci) {
-        const int c = c_lo + ci, cur = ci & 1;
-        if (ci + 1 < kChunksPerGroup) {
+      for (int c = 0; c < 4; ++c) {
+        const int cur = c & 1;
+        if (c + 1 < 4) {
           tmem_ld16_async(cs + 16 * (c + 1), sb[cur ^ 1]);
           tmem_ld16_async(cd + 16 * (c + 1), db[cur ^ 1]);
         }
         uint32_t pk[8], dk[8];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int c0 = kHalf * hh + 16 * c + 4 * q4;  // query column in the block
+          const int c0 = 64 * hc + 16 * c + 4 * q4;  // query column in the block
           const float4 l2 = *reinterpret_cast<const float4*>(stat + c0);
           const float4 dr = *reinterpret_cast<const float4*>(stat + kBT + c0);
           const float lv[4] = {l2.x, l2.y, l2.z, l2.w}, dv[4] = {dr.x, dr.y, dr.z, dr.w};
@@ -731,26 +781,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           dk[2 * q4] = pack2<kFp16>(dsv[0], dsv[1]);
           dk[2 * q4 + 1] = pack2<kFp16>(dsv[2], dsv[3]);
         }
-        tmem_st8(cs + packed_col(c), pk);  // P^T over S^T columns this group has already read
-        tmem_st8(cd + packed_col(c), dk);  // dS^T over dP^T columns this group has already read
-        if (ci + 1 < kChunksPerGroup) tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+        // dS^T and P^T over the dP^T columns of this chunk, which this warp has read (ds_col_dkdv)
+        tmem_st8(cd + 16 * c, dk);
+        tmem_st8(cd + 16 * c + 8, pk);
+        if (c + 1 < 4) {
+          tmem_wait_ld_pair(sb[cur ^ 1], db[cur ^ 1]);
+          if (c == 2) {  // all of this warp's S^T columns are in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->s_read);
+          }
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[hh]);
+      if (lane == 0) mbar_arrive(&bars->p_full);
     }
     if (ok) ok = warp_wait(&bars->o_done, 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       const size_t row = (static_cast<size_t>(u.k_row0 + min(kj, Lk - 1)) * p.H + h) * D;
-      // warps of half 0 store dV, those of half 1 dK, each column group its share of the 32-column chunks
-      const int ch_lo = cg * (D / 32) / kCG, ch_hi = (cg + 1) * (D / 32) / kCG;
-      if (hh == 0)
-        store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + kColA, 1.f, kj < Lk, p.status, p.g1_n, ch_lo, ch_hi);
-      else
-        store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + kColA + D, p.scale, kj < Lk, p.status, p.g0_n, ch_lo,
-                                          ch_hi);
+      constexpr uint32_t col_acc = C::template kColAcc<true>;
+      // warps of column half 0 store dV, those of half 1 dK
+      if (hc == 0) store_grad_row<D, kFp16, kOutF32>(p.g1, row, lane_base + col_acc, 1.f, kj < Lk, p.status, p.g1_n);
+      else store_grad_row<D, kFp16, kOutF32>(p.g0, row, lane_base + col_acc + D, p.scale, kj < Lk, p.status, p.g0_n);
     }
   }
   bwd_teardown(bars, warp, tbase);
@@ -758,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool kFp16, bool kOutF32>
 int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, cudaStream_t stream) {
-  const int smem = BwdCfg<D>::kSmemBytes;
+  const int smem = BwdCfg<D>::kSmemBytes, smem_q = BwdCfg<D>::kDqSmemBytes;
   const bool varlen = a.cu_seqlens != nullptr;
   const size_t rows = static_cast<size_t>(varlen ? 1 : a.B) * a.Nq * a.H;
   // varlen rows are those of one batch item of Nq = total rows: Drow [H, total]
@@ -770,7 +825,7 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   static PerContext<int> configured;
   int unused = 0;
   const int ce = configured.get(&unused, [&](int*) {
-    cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     return static_cast<int>(e);
   });
@@ -781,7 +836,7 @@ int launch_bwd_t(const BackwardArgs& a, const CUtensorMap (&m)[4], BwdParams p, 
   // dense: tiles per (b, h); varlen: slots per head, enough for the sum over the sequences of
   // ceil(len / 128) <= total / 128 + B (spare slots exit at once)
   pq.num_tiles = varlen ? a.Nq / kBT + a.B : (a.Nq + kBT - 1) / kBT;
-  kq<<<static_cast<unsigned>(pq.num_tiles * (varlen ? 1 : a.B) * a.H), kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], pq);
+  kq<<<static_cast<unsigned>(pq.num_tiles * (varlen ? 1 : a.B) * a.H), kThreads, smem_q, stream>>>(m[0], m[1], m[2], m[3], pq);
   BwdParams pk = p;
   pk.g0 = a.dk;
   pk.g1 = a.dv;
