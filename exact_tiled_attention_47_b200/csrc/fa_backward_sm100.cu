@@ -70,6 +70,9 @@ struct BwdCfg {
   // dQ(j) may still read K(j)), V three deep at D = 64 and two at D = 128, where shared memory ends
   // (V is read only by dP, which runs two blocks ahead; two V slots measured 2.6 % slower at D = 64)
   static constexpr int kKSt = 3, kVSt = (D == 64) ? 3 : 2;
+  // rings of equal depth: the release of K(j) after dQ(j) also releases V(j) (dP(j) completed before
+  // dQ(j) in the issuing thread's order), which saves one commit -- an MMA-pipe instruction -- per block
+  static constexpr bool kJointKV = kKSt == kVSt;
   static constexpr int kDqUsed = (2 + kKSt + kVSt) * kTileBytes + 256 + 1024;
   static constexpr int kDqSmemBytes = kDqUsed > 120 * 1024 ? kDqUsed : 120 * 1024;
 };
@@ -408,7 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d_hint(&tm_k, &bars->k_full[ks], sK(ks) + pn * kPanelBytes, pn * 64, h, u.k_row0 + j * kBT, keep);
         k_issued = j + 1;
-        if (!(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVSt) & 1) ^ 1, abort_flag, p.status))) break;
+        if (!C::kJointKV && !(ok = mbar_wait(&bars->v_empty[vs], ((j / C::kVSt) & 1) ^ 1, abort_flag, p.status)))
+          break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_S = [&](int jb) { mma_kk<D>(tbase + kColS, d_q, d_k + slot_off(jb % C::kKSt), idesc_s); };
       auto issue_dP = [&](int jb) {  // V(jb) is released once this product has completed
         mma_kk<D>(tbase + kColDP + 128 * (jb & 1), d_do, d_v + slot_off(jb % C::kVSt), idesc_s);
-        mma_commit(&bars->v_empty[jb % C::kVSt]);
+        if (!C::kJointKV) mma_commit(&bars->v_empty[jb % C::kVSt]);
       };
       bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) && wait_k(0) && wait_v(0);
       if (ok) {
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         mma_tn<ds_col_dq>(tbase + col_acc, tbase + kColDP + 128 * (j & 1), d_kn + slot_off(j % C::kKSt), idesc_g,
                           j > 0);
-        mma_commit(&bars->k_empty[j % C::kKSt]);  // K(j): S(j) and dQ(j) issued
+        mma_commit(&bars->k_empty[j % C::kKSt]);  // K(j): S(j) and dQ(j) issued (and V(j) with joint rings)
         if (j + 2 < n) {
           if (!(ok = wait_v(j + 2))) break;
           tc_fence_after();
