@@ -20,10 +20,10 @@
 //                       the dP^T columns they have read, then dV += P^T dO_i and dK += dS^T Q_i
 //                       accumulate in TMEM.  dV and dK * scale are written at the end.
 // Both recompute S and dP (two more GEMMs than the minimum) so that each gradient is owned by one
-// CTA and accumulates in TMEM.  Warp 8 is the TMA producer; warp 9 owns TMEM and issues every
-// tcgen05.mma from one thread.  A single thread issues an MMA about every 64 cycles whatever N up
-// to 128 (measured), so S and dP are whole-block products (M = N = 128) and the schedule keeps the
-// issue thread off the compute warps' path: S is released for the next block's S as soon as the
+// CTA and accumulates in TMEM.  Warp 8 is the TMA producer; warp 9 owns TMEM and issues S and dP
+// (and dV) from one thread, warp 10 the products that read dS (dQ; dK).  A single thread issues an
+// MMA about every 64 cycles whatever N up to 128 (measured), so S and dP are whole-block products
+// (M = N = 128) and the schedule keeps the issue threads off the compute warps' path: S is released for the next block's S as soon as the
 // compute warps hold it in registers, and dP goes into one of two TMEM buffers two blocks ahead
 // (after the gradient products that read that buffer; with one buffer, as in dK/dV at D = 128,
 // right after them).  The MMA forms are those of the forward kernel: SS with both operands K-major
@@ -42,9 +42,18 @@ namespace fa {
 namespace {
 
 constexpr int kBT = 128;  // rows per tile (queries or keys)
-constexpr int kThreads = 320;  // 8 compute warps, a TMA producer warp, an MMA warp
+// MMA-issuing threads: one issues S and dP (and owns TMEM); with two, a second issues the gradient
+// products that read the compute warps' results (dQ; dK), since one thread issues an MMA only every
+// ~64 cycles (two: +2 % at D = 128, no change at D = 64, measured)
+#ifndef FA_BWD_ISSUERS
+#define FA_BWD_ISSUERS 2
+#endif
+constexpr int kIssuers = FA_BWD_ISSUERS;
+static_assert(kIssuers == 1 || kIssuers == 2, "one or two MMA issuers");
+constexpr int kThreads = (9 + kIssuers) * 32;  // 8 compute warps, a TMA producer warp, the MMA warps
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;   // S and dP (and, with one issuer, everything); owns TMEM
+constexpr int kMmaWarp2 = 10;  // with two issuers: the gradient products that read dS (dQ; dK)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPanelBytes = kBT * 64 * 2;  // one 64-column (128-byte) swizzle panel of a tile
 constexpr int kMaxStages = 3;  // streamed-tile stages: 3 at D = 64, 2 at D = 128 (shared memory)
@@ -158,7 +167,8 @@ struct BwdBars {
   uint64_t s_full;   // S and dP of the next block are in TMEM (one phase per block)
   uint64_t s_read;   // the compute warps hold the block's S in registers: S may be overwritten
   uint64_t p_full;   // the block's packed dS (and P^T) are in TMEM
-  uint64_t o_done, drain;
+  uint64_t o_done, drain, drain2;
+  uint64_t g_done[2];  // two issuers: the block's dS-reading product (dQ; dK) has completed
   uint32_t tmem_base;
   int abort_flag;
   int unit_b, unit_t;
@@ -304,17 +314,18 @@ __device__ __forceinline__ void store_grad_row(void* out, size_t row_elem, uint3
   }
 }
 
-__device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
+// o_done_count: the issuing threads whose products accumulate into the CTA's gradients
+__device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp, int o_done_count) {
   if (threadIdx.x == 0) {
     mbar_init(&bars->fixed_full, 1);
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&bars->st_full[s], 1);
-      mbar_init(&bars->st_empty[s], 1);
+      mbar_init(&bars->st_empty[s], kIssuers);  // every issuing thread reads the streamed stage
       mbar_init(&bars->stat_full[s], 1);
     }
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->k_empty[s], kIssuers);  // K: S (first thread) and dQ (second thread)
     }
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bars->v_full[s], 1);
@@ -323,8 +334,11 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_read, 8);
     mbar_init(&bars->p_full, 8);
-    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_done, o_done_count);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain2, 1);
+    mbar_init(&bars->g_done[0], 1);
+    mbar_init(&bars->g_done[1], 1);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -388,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return;
   }
-  bwd_setup(bars, warp);
+  bwd_setup(bars, warp, 1);
   const uint32_t tbase = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
 
@@ -425,27 +439,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = max(0, v_issued - C::kVSt); j < v_issued; ++j) drain_wait(&bars->v_full[j % C::kVSt], (j / C::kVSt) & 1);
       }
     }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      // Block j: S = Q K_j^T into the S columns and dP = dO V_j^T into dP buffer j % 2 (N = 128, so
-      // each MMA carries twice the work of a half block at the same issue cost), then, once the
-      // compute warps have packed dS into that buffer, dQ += dS K_j.  S(j+1) is issued as soon as the
-      // compute warps hold S(j) in registers; dP(j+2) goes into buffer j % 2 right after dQ(j), so
-      // only S is issued between the blocks of the compute warps.
-      constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
-      constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
-      constexpr uint32_t col_acc = C::template kColAcc<false>;
-      const uint64_t d_q = desc_kmajor(sQ), d_do = desc_kmajor(sDO);
-      const uint64_t d_k = desc_kmajor(sK(0)), d_v = desc_kmajor(sV(0)), d_kn = desc_nmajor(sK(0));
-      auto slot_off = [&](int slot) { return static_cast<uint64_t>((slot * C::kTileBytes) >> 4); };
-      auto wait_k = [&](int jb) {
-        return mbar_wait(&bars->k_full[jb % C::kKSt], (jb / C::kKSt) & 1, abort_flag, p.status);
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+    // Block j: S = Q K_j^T into the S columns and dP = dO V_j^T into dP buffer j % 2 (N = 128, so
+    // each MMA carries twice the work of a half block at the same issue cost), then, once the compute
+    // warps have packed dS into that buffer, dQ += dS K_j.  S(j+1) is issued as soon as the compute
+    // warps hold S(j) in registers; dP(j+2) goes into buffer j % 2 once dQ(j) no longer needs it, so
+    // only S is issued between the blocks of the compute warps.  With two issuing threads the second
+    // issues dQ (and reports its completion: g_done), so the two streams of MMAs are issued side by
+    // side.
+    constexpr int fmt = kFp16 ? 0 : 1;
+    constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+    constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+    constexpr uint32_t col_acc = C::template kColAcc<false>;
+    const uint64_t d_q = desc_kmajor(sQ), d_do = desc_kmajor(sDO);
+    const uint64_t d_k = desc_kmajor(sK(0)), d_v = desc_kmajor(sV(0)), d_kn = desc_nmajor(sK(0));
+    auto slot_off = [&](int slot) { return static_cast<uint64_t>((slot * C::kTileBytes) >> 4); };
+    auto wait_k = [&](int jb) {
+      return mbar_wait(&bars->k_full[jb % C::kKSt], (jb / C::kKSt) & 1, abort_flag, p.status);
+    };
+    auto wait_v = [&](int jb) {
+      return mbar_wait(&bars->v_full[jb % C::kVSt], (jb / C::kVSt) & 1, abort_flag, p.status);
+    };
+    auto issue_dQ = [&](int j) {
+      mma_tn<ds_col_dq>(tbase + col_acc, tbase + kColDP + 128 * (j & 1), d_kn + slot_off(j % C::kKSt), idesc_g,
+                        j > 0);
+    };
+    if (lane == 0 && warp == kMmaWarp) {
+      auto issue_S = [&](int jb) {
+        mma_kk<D>(tbase + kColS, d_q, d_k + slot_off(jb % C::kKSt), idesc_s);
+        // with two issuers this thread's share of releasing block jb's slots: S(jb), and dP(jb)
+        // issued before it
+        if (kIssuers == 2) mma_commit(&bars->k_empty[jb % C::kKSt]);
       };
-      auto wait_v = [&](int jb) {
-        return mbar_wait(&bars->v_full[jb % C::kVSt], (jb / C::kVSt) & 1, abort_flag, p.status);
-      };
-      auto issue_S = [&](int jb) { mma_kk<D>(tbase + kColS, d_q, d_k + slot_off(jb % C::kKSt), idesc_s); };
       auto issue_dP = [&](int jb) {  // V(jb) is released once this product has completed
         mma_kk<D>(tbase + kColDP + 128 * (jb & 1), d_do, d_v + slot_off(jb % C::kVSt), idesc_s);
         if (!C::kJointKV) mma_commit(&bars->v_empty[jb % C::kVSt]);
@@ -453,8 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
-        issue_S(0);
         issue_dP(0);
+        issue_S(0);
         mma_commit(&bars->s_full);
         if (n > 1 && (ok = wait_v(1))) {
           tc_fence_after();
@@ -469,20 +494,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_S(j + 1);
           mma_commit(&bars->s_full);  // S(j+1) and dP(j+1)
         }
-        if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        mma_tn<ds_col_dq>(tbase + col_acc, tbase + kColDP + 128 * (j & 1), d_kn + slot_off(j % C::kKSt), idesc_g,
-                          j > 0);
-        mma_commit(&bars->k_empty[j % C::kKSt]);  // K(j): S(j) and dQ(j) issued (and V(j) with joint rings)
+        if (kIssuers == 1) {
+          if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_dQ(j);
+          mma_commit(&bars->k_empty[j % C::kKSt]);  // K(j): S(j) and dQ(j) issued (and V(j) with joint rings)
+        }
         if (j + 2 < n) {
+          // dP(j+2) goes into buffer j % 2: after dQ(j) in this thread's order, or once the other
+          // thread's dQ(j) has completed
+          if (kIssuers == 2 && !(ok = mbar_wait(&bars->g_done[j & 1], (j >> 1) & 1, abort_flag, p.status))) break;
           if (!(ok = wait_v(j + 2))) break;
           tc_fence_after();
-          issue_dP(j + 2);  // into buffer j % 2, after dQ(j) (the tensor core keeps one thread's order)
+          issue_dP(j + 2);
         }
       }
-      if (ok) mma_commit(&bars->o_done);
+      if (kIssuers == 1 && ok) mma_commit(&bars->o_done);
       mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
+    } else if (kIssuers == 2 && lane == 0 && warp == kMmaWarp2) {
+      bool ok = true;
+      for (int j = 0; ok && j < n; ++j) {
+        if (!(ok = mbar_wait(&bars->p_full, j & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_dQ(j);
+        mma_commit(&bars->g_done[j & 1]);         // buffer j % 2 may take dP(j+2)
+        mma_commit(&bars->k_empty[j % C::kKSt]);  // this thread's share of releasing K(j) (and V(j))
+      }
+      if (ok) mma_commit(&bars->o_done);
+      mma_commit(&bars->drain2);
+      drain_wait(&bars->drain2, 0);
     }
   } else {
     const int hc = warp >> 2;  // column half of every key block this warp works on
@@ -611,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return;
   }
-  bwd_setup(bars, warp);
+  bwd_setup(bars, warp, kIssuers);
   const uint32_t tbase = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
 
@@ -666,31 +707,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bars->fixed_full, 0);
       for (int jj = max(0, issued - C::kSt); jj < issued; ++jj) drain_wait(&bars->st_full[jj % C::kSt], (jj / C::kSt) & 1);
     }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      // Query block i (jj-th of the tile): S^T = K Q_i^T into the S columns and dP^T = V dO_i^T into a
-      // dP buffer (N = 128); once the compute warps have packed dS^T and P^T into that buffer,
-      // dV += P^T dO_i and dK += dS^T Q_i.  S^T(jj+1) is issued as soon as the compute warps hold
-      // S^T(jj) in registers.  With two dP buffers (D = 64) dP^T(jj+2) follows the products of block
-      // jj; with one (D = 128) dP^T(jj+1) does.
-      constexpr int fmt = kFp16 ? 0 : 1;
-      constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
-      constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
-      constexpr int kBufs = C::template kDPBufs<true>;
-      constexpr uint32_t col_acc = C::template kColAcc<true>;
-      const uint64_t d_k = desc_kmajor(sK), d_v = desc_kmajor(sV);
-      const uint64_t d_q = desc_kmajor(sQ(0)), d_do = desc_kmajor(sDO(0));
-      const uint64_t d_qn = desc_nmajor(sQ(0)), d_don = desc_nmajor(sDO(0));
-      auto stage_off = [&](int st) { return static_cast<uint64_t>((st * C::kTileBytes) >> 4); };
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+    // Query block i (jj-th of the tile): S^T = K Q_i^T into the S columns and dP^T = V dO_i^T into a
+    // dP buffer (N = 128); once the compute warps have packed dS^T and P^T into that buffer,
+    // dV += P^T dO_i and dK += dS^T Q_i.  S^T(jj+1) is issued as soon as the compute warps hold
+    // S^T(jj) in registers.  With two dP buffers (D = 64) dP^T(jj+2) follows the products of block
+    // jj; with one (D = 128) dP^T(jj+1) does.  With two issuing threads the second issues dK (and
+    // reports its completion: g_done) while the first issues S^T, dP^T and dV.
+    constexpr int fmt = kFp16 ? 0 : 1;
+    constexpr uint32_t idesc_s = instr_desc_f16(kBT, kBT, fmt, 0);
+    constexpr uint32_t idesc_g = instr_desc_f16(kBT, D, fmt, 1);
+    constexpr int kBufs = C::template kDPBufs<true>;
+    constexpr uint32_t col_acc = C::template kColAcc<true>;
+    const uint64_t d_k = desc_kmajor(sK), d_v = desc_kmajor(sV);
+    const uint64_t d_q = desc_kmajor(sQ(0)), d_do = desc_kmajor(sDO(0));
+    const uint64_t d_qn = desc_nmajor(sQ(0)), d_don = desc_nmajor(sDO(0));
+    auto stage_off = [&](int st) { return static_cast<uint64_t>((st * C::kTileBytes) >> 4); };
+    auto buf = [&](int jb) { return kColDP + 128 * (jb % kBufs); };
+    // dP^T of block jb + kBufs goes out after block jb's products: it needs block jb + kBufs's stage
+    // (kSt >= kBufs + 1 stages, so it is not block jb's own)
+    static_assert(C::kSt >= kBufs + 1, "stages for the dP lookahead");
+    if (lane == 0 && warp == kMmaWarp) {
       auto wait_stage = [&](int jb) {
         return mbar_wait(&bars->st_full[jb % C::kSt], (jb / C::kSt) & 1, abort_flag, p.status);
       };
-      auto buf = [&](int jb) { return kColDP + 128 * (jb % kBufs); };
       auto issue_S = [&](int jb) { mma_kk<D>(tbase + kColS, d_k, d_q + stage_off(jb % C::kSt), idesc_s); };
       auto issue_dP = [&](int jb) { mma_kk<D>(tbase + buf(jb), d_v, d_do + stage_off(jb % C::kSt), idesc_s); };
-      // dP^T of block jb + kBufs goes out after block jb's products: it needs block jb + kBufs's stage
-      // (kSt >= kBufs + 1 stages, so it is not block jb's own)
-      static_assert(C::kSt >= kBufs + 1, "stages for the dP lookahead");
       bool ok = mbar_wait(&bars->fixed_full, 0, abort_flag, p.status) && wait_stage(0);
       if (ok) {
         tc_fence_after();
@@ -717,20 +759,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!(ok = mbar_wait(&bars->p_full, jj & 1, abort_flag, p.status))) break;
         tc_fence_after();
-        // dV += P^T dO_i,  dK += dS^T Q_i  (P^T 8 columns after dS^T in every chunk)
-        mma_tn2<ds_col_dkdv>(tbase + col_acc, tbase + buf(jj) + 8, d_don + stage_off(st), tbase + col_acc + D,
-                             tbase + buf(jj), d_qn + stage_off(st), idesc_g, jj > 0);
-        mma_commit(&bars->st_empty[st]);  // every product reading stage st is issued
+        if (kIssuers == 1) {
+          // dV += P^T dO_i,  dK += dS^T Q_i  (P^T 8 columns after dS^T in every chunk)
+          mma_tn2<ds_col_dkdv>(tbase + col_acc, tbase + buf(jj) + 8, d_don + stage_off(st), tbase + col_acc + D,
+                               tbase + buf(jj), d_qn + stage_off(st), idesc_g, jj > 0);
+        } else {
+          mma_tn<ds_col_dkdv>(tbase + col_acc, tbase + buf(jj) + 8, d_don + stage_off(st), idesc_g, jj > 0);
+        }
+        mma_commit(&bars->st_empty[st]);  // this thread's products reading stage st are issued
         if (jj + kBufs < n) {
+          // dP^T(jj+kBufs) goes into block jj's buffer: after its products in this thread's order, or
+          // once the other thread's dK(jj) has completed
+          if (kIssuers == 2 && !(ok = mbar_wait(&bars->g_done[jj % kBufs], (jj / kBufs) & 1, abort_flag, p.status)))
+            break;
           if (!(ok = wait_stage(jj + kBufs))) break;
           tc_fence_after();
-          issue_dP(jj + kBufs);  // into block jj's buffer, after its products (the tensor core keeps order)
+          issue_dP(jj + kBufs);
           if (kBufs == 1) mma_commit(&bars->s_full);  // S^T(jj+1) and dP^T(jj+1)
         }
       }
       if (ok) mma_commit(&bars->o_done);
       mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
+    } else if (kIssuers == 2 && lane == 0 && warp == kMmaWarp2) {
+      bool ok = true;
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const int st = jj % C::kSt;
+        if (!(ok = mbar_wait(&bars->p_full, jj & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        mma_tn<ds_col_dkdv>(tbase + col_acc + D, tbase + buf(jj), d_qn + stage_off(st), idesc_g, jj > 0);  // dK
+        mma_commit(&bars->g_done[jj % kBufs]);  // block jj's buffer may take dP^T(jj + kBufs)
+        mma_commit(&bars->st_empty[st]);        // this thread's share of releasing stage st
+      }
+      if (ok) mma_commit(&bars->o_done);
+      mma_commit(&bars->drain2);
+      drain_wait(&bars->drain2, 0);
     }
   } else {
     constexpr int kBufs = C::template kDPBufs<true>;
