@@ -60,11 +60,13 @@ def test_token_rates():
     line = {"ms_per_step": 2.0, "config": {"B": 4, "N": 8192},
             "decode": {"ms_per_step": 1.0, "config": {"B": 64},
                        "gqa": {"ms_per_step": 0.5, "config": {"B": 64}},
+                       "paged": {"ms_per_step": 0.25, "config": {"B": 64}},
                        "sharded": {"ms_per_step": 4.0, "config": {"B": 4}}}}
     bench.add_token_rates(line, 2)
     assert line["tokens_per_s"] == 4 * 8192 * 2 / 2e-3
     assert line["decode"]["tokens_per_s"] == 64 * 2 / 1e-3
     assert line["decode"]["gqa"]["tokens_per_s"] == 64 * 2 / 0.5e-3
+    assert line["decode"]["paged"]["tokens_per_s"] == 64 * 2 / 0.25e-3  # every rank its own batch
     assert line["decode"]["sharded"]["tokens_per_s"] == 4 / 4e-3  # one problem over the ranks
     # partial lines (a leg switched off) keep working
     for partial in ({"ms_per_step": None, "config": {}, "decode": None}, {"decode": {"ms_per_step": 1.0}}, {}):
