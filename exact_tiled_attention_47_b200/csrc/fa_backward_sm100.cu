@@ -264,6 +264,15 @@ __host__ __device__ constexpr uint32_t ds_col_dkdv(int kk) {
   return static_cast<uint32_t>(64 * (kk >> 2) + 16 * (kk & 3));
 }
 
+// packed product of fp32 pairs; with fma.rn.f32x2 and add.rn.f32x2 it rounds each lane as the scalar
+// instruction does (round to nearest, subnormals kept), at one issue slot per pair
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_of(const uint32_t* x) { return f2(__uint_as_float(x[0]), __uint_as_float(x[1])); }
+
 // d (+)= A (TMEM, 128 x 128 packed 16-bit, chunk kk at a_tmem + col(kk)) * B (shared, N-major 128
 // rows from the descriptor b; 16 rows = two 8-row swizzle atoms = 2048 bytes).  Two products
 // (d0, d1) have their K steps interleaved.
@@ -542,6 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lse2 = (qi < Lq && lse != -INFINITY) ? lse * kLog2e : INFINITY;
     const float dr = (qi < Lq && stat_in) ? p.drow[stat] : 0.f;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2(sl2, sl2), nlse2x2 = f2(-lse2, -lse2), ndrx2 = f2(-dr, -dr);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       if (!(ok = warp_wait(&bars->s_full, j & 1, abort_flag, p.status))) break;
@@ -565,13 +575,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int c0 = 64 * hc + 16 * c + 2 * i;  // key column in the block
-          float p0 = ex2(fmaf(__uint_as_float(sb[cur][2 * i]), sl2, -lse2));
-          float p1 = ex2(fmaf(__uint_as_float(sb[cur][2 * i + 1]), sl2, -lse2));
+          // P = 2^(s scale log2e - LSE log2e), dS = P (dP - Drow), two columns per instruction
+          float x0, x1;
+          f2_split(f2_fma(f2_of(&sb[cur][2 * i]), sl2x2, nlse2x2), x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
           if (masked) {
             if (c0 >= lim) p0 = 0.f;
             if (c0 + 1 >= lim) p1 = 0.f;
           }
-          pk[i] = pack2<kFp16>(p0 * (__uint_as_float(db[cur][2 * i]) - dr), p1 * (__uint_as_float(db[cur][2 * i + 1]) - dr));
+          float d0, d1;
+          f2_split(f2_mul(f2(p0, p1), f2_add(f2_of(&db[cur][2 * i]), ndrx2)), d0, d1);
+          pk[i] = pack2<kFp16>(d0, d1);
         }
         tmem_st8(cd + 8 * c, pk);  // dS over dP columns this warp has already read (ds_col_dq)
         if (c + 1 < 4) {
@@ -616,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + C::kTileBytes;
   auto sQ = [&](int st) { return smem + (2 + st) * C::kTileBytes; };
   auto sDO = [&](int st) { return smem + (2 + C::kSt + st) * C::kTileBytes; };
-  float* sStat = reinterpret_cast<float*>(smem + (2 + 2 * C::kSt) * C::kTileBytes);  // [stage][lse2 | drow][128]
+  float* sStat = reinterpret_cast<float*>(smem + (2 + 2 * C::kSt) * C::kTileBytes);  // [stage][-lse2 | -drow][128]
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + (2 + 2 * C::kSt) * C::kTileBytes + 2 * C::kSt * kBT * 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -680,8 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       issued = jj + 1;
-      // the block's LSE (log2 units; +inf for rows without keys or past the end, so P = 0) and Drow:
-      // all eight loads of a lane are independent and in flight together
+      // the block's negated LSE (log2 units; -inf for rows without keys or past the end, so P = 0) and
+      // negated Drow: all eight loads of a lane are independent and in flight together
       float* stat = sStat + st * 2 * kBT;
       // LSE and Drow: [B, H, Nq] dense, [H, total] varlen
       const size_t base = p.cu == nullptr ? (static_cast<size_t>(b) * p.H + h) * p.Nq
@@ -697,8 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        stat[lane + 32 * e] = (lv[e] != -INFINITY) ? lv[e] * kLog2e : INFINITY;
-        stat[kBT + lane + 32 * e] = dv[e];
+        stat[lane + 32 * e] = (lv[e] != -INFINITY) ? -(lv[e] * kLog2e) : -INFINITY;
+        stat[kBT + lane + 32 * e] = -dv[e];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->stat_full[st]);  // release: orders the warp's stores above
@@ -802,6 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kj = n0 + r;  // this thread's key
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       const int i = i_first + jj, st = jj % C::kSt;
@@ -832,16 +847,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int c0 = 64 * hc + 16 * c + 4 * q4;  // query column in the block
-          const float4 l2 = *reinterpret_cast<const float4*>(stat + c0);
-          const float4 dr = *reinterpret_cast<const float4*>(stat + kBT + c0);
-          const float lv[4] = {l2.x, l2.y, l2.z, l2.w}, dv[4] = {dr.x, dr.y, dr.z, dr.w};
+          // the four queries' -LSE log2e and -Drow as pairs
+          const ulonglong2 nl = *reinterpret_cast<const ulonglong2*>(stat + c0);
+          const ulonglong2 nd = *reinterpret_cast<const ulonglong2*>(stat + kBT + c0);
+          const uint64_t nlv[2] = {nl.x, nl.y}, ndv[2] = {nd.x, nd.y};
           float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float pe = ex2(fmaf(__uint_as_float(sb[cur][4 * q4 + e]), sl2, -lv[e]));
-            if (masked && c0 + e < q_lo) pe = 0.f;
-            pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(db[cur][4 * q4 + e]) - dv[e]);
+          for (int e = 0; e < 4; e += 2) {
+            // P = 2^(s scale log2e - LSE log2e), dS = P (dP - Drow), two queries per instruction
+            float x0, x1;
+            f2_split(f2_fma(f2_of(&sb[cur][4 * q4 + e]), sl2x2, nlv[e / 2]), x0, x1);
+            pv[e] = ex2(x0);
+            pv[e + 1] = ex2(x1);
+            if (masked) {
+              if (c0 + e < q_lo) pv[e] = 0.f;
+              if (c0 + e + 1 < q_lo) pv[e + 1] = 0.f;
+            }
+            f2_split(f2_mul(f2(pv[e], pv[e + 1]), f2_add(f2_of(&db[cur][4 * q4 + e]), ndv[e / 2])), dsv[e], dsv[e + 1]);
           }
           pk[2 * q4] = pack2<kFp16>(pv[0], pv[1]);
           pk[2 * q4 + 1] = pack2<kFp16>(pv[2], pv[3]);
