@@ -51,6 +51,19 @@ MUTANTS = {
     "paged_partial_page_dropped": ("attention.py", "for i in range(-(-L // ps)):", "for i in range(L // ps):"),
     "paged_row_in_page": ("attention.py", "k_g[b, i * ps:(i + 1) * ps] = k_pages[page]",
                           "k_g[b, i * ps:(i + 1) * ps] = k_pages[page][::-1]"),
+    "gqa_head_modulo": ("attention.py", "k_cache[b, :L, h // G, :], v_cache[b, :L, h // G, :]",
+                        "k_cache[b, :L, h % Hkv, :], v_cache[b, :L, h % Hkv, :]"),
+    "varlen_key_offset": ("attention.py", "k[s0:s1, h, :]", "k[:s1 - s0, h, :]"),
+    "padded_mask_on_queries": ("attention.py", "s = np.where(kv[None, :], s, -np.inf)",
+                               "s = np.where(kv[:, None], s, -np.inf)"),
+    "split_floor": ("online.py", "per = -(-nk // num_splits)", "per = max(1, nk // num_splits)"),
+    "split_lse_without_max": ("online.py", "lse[s] = m + math.log(l)", "lse[s] = math.log(l)"),
+    "tiled_l_not_rescaled": ("online.py", "l = alpha * l + p.sum(axis=1)", "l = l + p.sum(axis=1)"),
+    "tiled_causal_top_left": ("online.py", "cols[None, :] <= rows[:, None] + (nk - nq)", "cols[None, :] <= rows[:, None]"),
+    "bwd_dv_untransposed": ("backward.py", "dv = p.T @ do",
+                            "dv = (p @ do)[: v.shape[0]] if p.shape[0] >= v.shape[0] else p.T @ do"),
+    "bwd_varlen_key_offset": ("backward.py", "q[s0:s1, h], k[s0:s1, h], v[s0:s1, h]",
+                              "q[s0:s1, h], k[:s1 - s0, h], v[s0:s1, h]"),
 }
 
 
